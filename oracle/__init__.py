@@ -1,0 +1,11 @@
+"""Plain fp64 CPU oracle for the dynamic block-sparse attention path.
+
+Test infrastructure only: imported by ``tests/``, ``__graft_entry__.smoke()``
+and the CPU-baseline leg of ``bench.py``; never by the product path.
+"""
+from .sparse_attn_ref import *  # noqa: F401,F403
+from .sparse_attn_ref import (BLOCK, E4M3_MAX, attn_int8fp8_from_codes, attn_ref_exact,  # noqa: F401
+                              attn_ref_int8fp8, block_means, block_scores, e4m3_decode,
+                              e4m3_encode, e4m3_round, keep_count, kth_threshold, max_abs_err,
+                              n_blocks, plan_mask, plan_ref, quant_qk_ref, quant_v_ref,
+                              rel_l1_err, select_topk)
