@@ -1,0 +1,154 @@
+/*
+ * lx_sparse_attn.h -- dynamic block-sparse, low-precision self-attention for
+ * long-sequence video DiTs, for NVIDIA B200 (sm_100a).
+ *
+ * What it computes (the method LightX2V calls Dynamic Sparse SageAttention):
+ *  - "600倍加速，720p视频实时生成！单卡也能带的动14B模型", §动态稀疏量化注意力:
+ *    the importance of attention tiles is estimated from block-level means of
+ *    Q and K, key blocks are chosen at run time, only the activated tiles are
+ *    computed and a chosen block stays dense inside (typical sparsity 80-90%).
+ *  - same page, §高效推理算子: about 10% of the blocks are kept and the
+ *    arithmetic is Q/K INT8 with V FP8.
+ *  - "Run Wan2.2-A14B on One RTX 5090: 720p Video in 3.8s", §3 Dynamic sparse
+ *    attention: the same in English (top 10-20% of blocks, dense inside).
+ * The pages fix no block size, score, selection rule or scale granularity;
+ * this library's fixed reading is: 64-token blocks (nB = ceil(L/64), the last
+ * block may be partial), score s[i][j] = mean(Q_i) . mean(K_j) / sqrt(D),
+ * keep k = clamp(ceil(keep*nB - 1e-6), 1, nB) key blocks per query block with
+ * ties to the lower index, INT8 Q/K with one absmax/127 scale per (b,h,block),
+ * FP8 E4M3 V with one absmax/448 scale per (b,h,channel), and in INT8/FP8
+ * mode P quantised to E4M3 (scale 448) against the running row max, one
+ * 64-key block at a time in ascending key-block order.
+ *
+ * Conventions for every entry point:
+ *  - All tensors are device memory owned by the caller; the library allocates
+ *    no memory and keeps no state besides one status word per device.
+ *  - Q, K, V, O are bf16 [B,H,L,D] with element strides sB, sH, sL (the stride
+ *    of D is 1); D is 64 or 128; base pointers and every stride in bytes must
+ *    be multiples of 16.
+ *  - Argument errors are detected on the host before any launch and return a
+ *    negative status; nothing is launched then.  Launches are asynchronous on
+ *    `stream`; a launch failure returns LX_ERR_CUDA.  Errors found on the device
+ *    (a bounded wait that ran out, a malformed plan) are recorded in the status
+ *    word and reported by lx_last_device_status().
+ *  - Calls are stream-ordered and never synchronise, except
+ *    lx_last_device_status().
+ */
+#ifndef LX_SPARSE_ATTN_H
+#define LX_SPARSE_ATTN_H
+
+#include <stddef.h>
+#include <stdint.h>
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define LX_BLOCK 64
+
+typedef enum lx_status {
+  LX_OK = 0,
+  LX_ERR_INVALID = -1,     /* bad pointer, shape, stride or keep */
+  LX_ERR_UNSUPPORTED = -2, /* D not in {64,128}, or nB beyond the planner limit */
+  LX_ERR_ALIGN = -3,       /* a pointer or byte stride not a multiple of 16 */
+  LX_ERR_WORKSPACE = -4,   /* workspace null or smaller than the size query says */
+  LX_ERR_CUDA = -5,        /* a CUDA call or launch failed */
+  LX_ERR_TIMEOUT = -6,     /* device: a bounded wait ran out (kernel gave up cleanly) */
+  LX_ERR_PLAN = -7         /* device: a plan row not strictly ascending / out of range, or non-finite scores */
+} lx_status;
+
+typedef enum lx_mode { LX_MODE_BF16 = 0, LX_MODE_INT8FP8 = 1 } lx_mode;
+
+/* A bf16 [B,H,L,D] tensor view; strides in elements, stride of D is 1. */
+typedef struct lx_bhld {
+  void* data;
+  int64_t B, H, L, D;
+  int64_t sB, sH, sL;
+} lx_bhld;
+
+/* A block plan.  idx: int32 [B,H,nB,k], each row the kept key-block ids in
+ * strictly ascending order.  mask: uint32 [B,H,nB,ceil(nB/32)], bit (j%32) of
+ * word j/32 set iff key block j is kept; may be NULL.  Plain caller-owned data:
+ * a caller may build or edit a plan by hand. */
+typedef struct lx_plan {
+  int32_t* idx;
+  uint32_t* mask;
+  int64_t B, H, L, nB, k;
+  int32_t block; /* always LX_BLOCK */
+} lx_plan;
+
+/* Sizes of a plan.  k = clamp(ceil(keep*nB - 1e-6), 1, nB) with nB = ceil(L/64);
+ * idx_bytes / mask_bytes size the plan arrays; ws_bytes sizes the workspace of
+ * lx_sparse_attn_plan (two fp32 [B,H,nB,D] block-mean arrays).
+ * keep must lie in (0, 1].  Any output pointer may be NULL. */
+lx_status lx_plan_size(int64_t B, int64_t H, int64_t L, int64_t D, double keep, int64_t* k, size_t* idx_bytes,
+                       size_t* mask_bytes, size_t* ws_bytes);
+
+/* Step a1 -- block means ("600倍加速…", §动态稀疏量化注意力: "块级均值").
+ * mq, mk: fp32 [B,H,nB,D] contiguous outputs, mean over the valid tokens of
+ * each 64-token block (the last block divides by its own token count). */
+lx_status lx_pool_means(const lx_bhld* Q, const lx_bhld* K, float* mq, float* mk, cudaStream_t stream);
+
+/* Step a2 -- score and select.  From the block means (layout as above) writes
+ * plan->idx (and plan->mask when not NULL): per query block the k key blocks
+ * with the largest mean(Q_i).mean(K_j)/sqrt(D), ties to the lower index,
+ * ascending.  plan->idx/mask must be set by the caller; the call fills
+ * plan->B, H, L, nB, k and block.  nB must not exceed 2432 (L <= 155648). */
+lx_status lx_score_topk(const float* mq, const float* mk, int64_t B, int64_t H, int64_t L, int64_t D, double keep,
+                        lx_plan* plan, cudaStream_t stream);
+
+/* Steps a1 + a2 -- the planner.  ws: at least ws_bytes of lx_plan_size. */
+lx_status lx_sparse_attn_plan(const lx_bhld* Q, const lx_bhld* K, double keep, lx_plan* plan, void* ws,
+                              size_t ws_bytes, cudaStream_t stream);
+
+/* Step a3 -- INT8 Q and K ("600倍加速…", §高效推理算子: "Q/K INT8").
+ * qc, kc: int8 [B,H,L,D] contiguous codes; qs, ks: fp32 [B,H,nB] scales.
+ * scale = absmax/127 over the block's valid tokens and all D channels (1 for
+ * an all-zero block); code = clamp(rint_even(fl32(x * fl32(127/absmax))), +-127). */
+lx_status lx_quantize_qk(const lx_bhld* Q, const lx_bhld* K, int8_t* qc, float* qs, int8_t* kc, float* ks,
+                         cudaStream_t stream);
+
+/* Step a3 -- FP8 E4M3 V ("600倍加速…", §高效推理算子: "V FP8").
+ * vc: uint8 [B,H,L,D] contiguous E4M3 codes; vs: fp32 [B,H,D] scales =
+ * absmax over all L tokens / 448 (1 for an all-zero channel);
+ * code = E4M3_rn_satfinite(fl32(v * fl32(448/absmax))).
+ * amax_ws: caller scratch of B*H*D uint32 (zeroed by the call). */
+lx_status lx_quantize_v(const lx_bhld* V, uint8_t* vc, float* vs, uint32_t* amax_ws, cudaStream_t stream);
+
+/* Step a4 -- attention over the kept blocks in BF16 (tcgen05 kind::f16).
+ * O[t] = sum_u softmax_u(q_t.k_u/sqrt(D)) v_u over the valid keys u of the
+ * kept blocks of t's query block ("600倍加速…", §动态稀疏量化注意力). */
+lx_status lx_attn_bf16(const lx_bhld* Q, const lx_bhld* K, const lx_bhld* V, const lx_plan* plan, const lx_bhld* O,
+                       cudaStream_t stream);
+
+/* Step a4 -- attention over the kept blocks from quantised operands
+ * (tcgen05 kind::i8 for QK^T, kind::f8f6f4 for PV).  qc, kc, vc, qs, ks, vs as
+ * written by lx_quantize_qk / lx_quantize_v for tensors of shape
+ * [B,H,L,D] = O's shape.  P follows the E4M3 protocol stated at the top. */
+lx_status lx_attn_int8fp8(const int8_t* qc, const float* qs, const int8_t* kc, const float* ks, const uint8_t* vc,
+                          const float* vs, const lx_plan* plan, const lx_bhld* O, cudaStream_t stream);
+
+/* Workspace of lx_sparse_attn_fwd: 0 for BF16; for INT8/FP8 the int8 Q/K codes,
+ * E4M3 V codes, their scales and the V absmax scratch (each 256-byte aligned). */
+lx_status lx_fwd_workspace_size(const lx_bhld* Q, lx_mode mode, size_t* bytes);
+
+/* Steps a3 + a4: O = sparse attention of (Q, K, V) under `plan` in `mode`. */
+lx_status lx_sparse_attn_fwd(const lx_bhld* Q, const lx_bhld* K, const lx_bhld* V, const lx_plan* plan, lx_mode mode,
+                             const lx_bhld* O, void* ws, size_t ws_bytes, cudaStream_t stream);
+
+/* Synchronises `stream`, returns and clears the device status word of the
+ * current device: LX_OK, LX_ERR_TIMEOUT, LX_ERR_PLAN, or LX_ERR_CUDA when the
+ * stream itself reports an error. */
+lx_status lx_last_device_status(cudaStream_t stream);
+
+/* Launches one kernel that waits on a barrier nothing completes, giving up
+ * after limit_ns; the failure path of every bounded wait, for tests. */
+lx_status lx_debug_wait_timeout(uint64_t limit_ns, cudaStream_t stream);
+
+const char* lx_status_string(lx_status status);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* LX_SPARSE_ATTN_H */

@@ -1,0 +1,110 @@
+"""Planner parity (steps a1 pool, a2 score + top-k) against the oracle."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import video_dit_dynamic_token_b200 as lx
+from video_dit_dynamic_token_b200 import synth
+from gpu_util import check_plan, to_np
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+
+def _inputs(B, H, L, d, seed=0, smooth=False):
+    if smooth:
+        raise NotImplementedError
+    return synth.random_qkv(B, H, L, d, seed=seed, device=DEV)
+
+
+@pytest.mark.parametrize("B,H,L,d", [(1, 2, 1024, 64), (1, 3, 1000, 128), (2, 2, 65, 128), (1, 1, 1, 64),
+                                     (1, 2, 130, 64)])
+def test_pool_means(B, H, L, d):
+    Q, K, _ = _inputs(B, H, L, d, seed=L)
+    mq, mk = lx.lx_pool_means(Q, K)
+    torch.cuda.synchronize()
+    for got, X in ((mq, Q), (mk, K)):
+        ref = oracle.block_means(X)
+        err = np.abs(to_np(got) - ref).max() / max(1e-30, np.abs(ref).max())
+        assert err < 2e-6, err
+
+
+def test_pool_means_strided_view():
+    # Wan's natural [B, L, H, D] layout, viewed as [B, H, L, D]
+    g = torch.Generator(device=DEV).manual_seed(1)
+    raw = torch.randn(2, 777, 3, 128, generator=g, device=DEV).to(torch.bfloat16)
+    Q = raw.permute(0, 2, 1, 3)
+    mq, mk = lx.lx_pool_means(Q, Q)
+    torch.cuda.synchronize()
+    ref = oracle.block_means(Q.contiguous())
+    assert np.abs(to_np(mq) - ref).max() < 2e-6 * np.abs(ref).max()
+
+
+@pytest.mark.parametrize("B,H,L,d,keep", [
+    (1, 2, 1024, 64, 0.25),      # the tiny workload shape
+    (1, 3, 1000, 128, 0.3),      # ragged last block
+    (2, 2, 4160, 128, 0.1),      # nB = 65 (odd), B = 2
+    (1, 2, 64, 128, 0.5),        # nB = 1
+    (1, 2, 65, 64, 0.5),         # last block of one token
+    (1, 1, 1, 64, 0.9),          # L = 1
+    (1, 2, 3000, 128, 1.0),      # keep everything
+    (1, 2, 3000, 128, 0.01),     # k = 1
+])
+def test_plan_parity_small(B, H, L, d, keep):
+    Q, K, _ = _inputs(B, H, L, d, seed=L + 7)
+    plan = lx.lx_sparse_attn_plan(Q, K, keep)
+    assert lx.lx_last_device_status() == 0
+    check_plan(plan.idx, plan.mask, Q.cpu(), K.cpu(), keep)
+
+
+def test_plan_parity_tiny_workload():
+    Q, K, _ = synth.make_workload("tiny")
+    plan = lx.lx_sparse_attn_plan(Q.to(DEV), K.to(DEV), 0.25)
+    assert lx.lx_last_device_status() == 0
+    check_plan(plan.idx, plan.mask, Q, K, 0.25)
+
+
+def test_plan_all_equal_scores_take_lowest_ids():
+    # zero Q: every score is 0, so the k lowest key ids must be kept
+    Q = torch.zeros(1, 1, 640, 128, dtype=torch.bfloat16, device=DEV)
+    _, K, _ = _inputs(1, 1, 640, 128, seed=3)
+    plan = lx.lx_sparse_attn_plan(Q, K, 0.3)
+    k = plan.k
+    assert np.array_equal(to_np(plan.idx)[0, 0], np.tile(np.arange(k), (10, 1)))
+
+
+def test_plan_duplicate_key_blocks_tie_to_lower_index():
+    Q, K, _ = _inputs(1, 1, 64 * 40, 128, seed=5)
+    K = K.clone()
+    K[0, 0, 64 * 30:64 * 31] = K[0, 0, 64 * 7:64 * 8]     # blocks 7 and 30 identical
+    K[0, 0, 64 * 33:64 * 34] = K[0, 0, 64 * 7:64 * 8]     # and 33
+    for keep in (0.05, 0.1, 0.2, 0.5):
+        plan = lx.lx_sparse_attn_plan(Q, K, keep)
+        check_plan(plan.idx, plan.mask, Q.cpu(), K.cpu(), keep)
+        gi = to_np(plan.idx)[0, 0]
+        for row in gi:   # a later duplicate is never kept without the earlier one
+            s = set(row.tolist())
+            assert not ((30 in s or 33 in s) and 7 not in s)
+            assert not (33 in s and 30 not in s)
+
+
+@pytest.mark.parametrize("name", ["480p", "720p", "long"])
+def test_plan_parity_full_size(name):
+    w = synth.WORKLOADS[name]
+    Q, K, _ = synth.make_qkv(w.B, w.H, w.d, w.grid, seed=0, device=DEV)
+    plan = lx.lx_sparse_attn_plan(Q, K, w.keep)
+    assert lx.lx_last_device_status() == 0
+    Qc, Kc = Q.cpu(), K.cpu()
+    del Q, K
+    check_plan(plan.idx, plan.mask, Qc, Kc, w.keep)
+
+
+@pytest.mark.parametrize("keep", [0.05, 0.5, 1.0])
+@pytest.mark.parametrize("smooth", [True, False])
+def test_plan_parity_720p_keep_sweep(keep, smooth):
+    w = synth.WORKLOADS["720p"]
+    Q, K, _ = synth.make_qkv(1, 4, w.d, w.grid, seed=1, smooth=smooth, device=DEV)
+    plan = lx.lx_sparse_attn_plan(Q, K, keep)
+    assert lx.lx_last_device_status() == 0
+    check_plan(plan.idx, plan.mask, Q.cpu(), K.cpu(), keep)

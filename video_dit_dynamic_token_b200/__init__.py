@@ -1,0 +1,213 @@
+"""Dynamic block-sparse, low-precision self-attention for video DiTs on B200.
+
+Thin Python binding over the C-ABI library ``liblx_sparse_attn.so`` (see
+``include/lx_sparse_attn.h``).  Functions carry the C names; they only marshal
+arguments: torch allocates device memory and supplies the current stream, and
+every step of the computation runs in the library's CUDA kernels.  There is no
+CPU fallback -- a missing library raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+from dataclasses import dataclass
+
+import torch
+
+from . import _abi
+from ._abi import LX_BLOCK, LX_MODE_BF16, LX_MODE_INT8FP8, LxBhld, LxPlan  # noqa: F401
+
+MODES = {"bf16": LX_MODE_BF16, "int8fp8": LX_MODE_INT8FP8}
+
+
+class LxError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        lib = _abi.load()
+        super().__init__(f"{where}: {lib.lx_status_string(status).decode()} (status {status})")
+        self.status = status
+
+
+def _check(status: int, where: str):
+    if status != 0:
+        raise LxError(status, where)
+
+
+def _stream(stream=None):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _ptr(t):
+    return ctypes.c_void_p(t.data_ptr()) if t is not None else None
+
+
+def bhld(t: torch.Tensor) -> LxBhld:
+    """View of a bf16 [B,H,L,D] CUDA tensor whose last dim is contiguous."""
+    if t.dtype != torch.bfloat16 or t.dim() != 4 or t.stride(3) != 1:
+        raise ValueError("expected a bf16 [B,H,L,D] tensor with contiguous D")
+    B, H, L, D = t.shape
+    sB, sH, sL, _ = t.stride()
+    return LxBhld(t.data_ptr(), B, H, L, D, sB, sH, sL)
+
+
+@dataclass
+class Plan:
+    """Kept-block plan: idx int32 [B,H,nB,k] ascending, mask uint32-bits [B,H,nB,W]."""
+    idx: torch.Tensor
+    mask: torch.Tensor | None
+    B: int
+    H: int
+    L: int
+    nB: int
+    k: int
+
+    def c(self) -> LxPlan:
+        return LxPlan(self.idx.data_ptr(), self.mask.data_ptr() if self.mask is not None else None,
+                      self.B, self.H, self.L, self.nB, self.k, LX_BLOCK)
+
+
+def lx_plan_size(B, H, L, D, keep):
+    lib = _abi.load()
+    k = ctypes.c_int64()
+    ib, mb, wb = ctypes.c_size_t(), ctypes.c_size_t(), ctypes.c_size_t()
+    _check(lib.lx_plan_size(B, H, L, D, float(keep), ctypes.byref(k), ctypes.byref(ib), ctypes.byref(mb),
+                            ctypes.byref(wb)), "lx_plan_size")
+    return k.value, ib.value, mb.value, wb.value
+
+
+def empty_plan(B, H, L, D, keep, device, with_mask=True) -> Plan:
+    k, _, _, _ = lx_plan_size(B, H, L, D, keep)
+    nB = (L + LX_BLOCK - 1) // LX_BLOCK
+    idx = torch.empty((B, H, nB, k), dtype=torch.int32, device=device)
+    mask = torch.empty((B, H, nB, (nB + 31) // 32), dtype=torch.int32, device=device) if with_mask else None
+    return Plan(idx, mask, B, H, L, nB, k)
+
+
+def lx_pool_means(Q, K, out=None, stream=None):
+    lib = _abi.load()
+    B, H, L, D = Q.shape
+    nB = (L + LX_BLOCK - 1) // LX_BLOCK
+    if out is None:
+        out = (torch.empty((B, H, nB, D), dtype=torch.float32, device=Q.device),
+               torch.empty((B, H, nB, D), dtype=torch.float32, device=Q.device))
+    q, k = bhld(Q), bhld(K)
+    _check(lib.lx_pool_means(ctypes.byref(q), ctypes.byref(k), _ptr(out[0]), _ptr(out[1]), _stream(stream)),
+           "lx_pool_means")
+    return out
+
+
+def lx_score_topk(mq, mk, L, keep, plan: Plan | None = None, stream=None) -> Plan:
+    lib = _abi.load()
+    B, H, nB, D = mq.shape
+    if plan is None:
+        plan = empty_plan(B, H, L, D, keep, mq.device)
+    cp = plan.c()
+    _check(lib.lx_score_topk(_ptr(mq), _ptr(mk), B, H, L, D, float(keep), ctypes.byref(cp), _stream(stream)),
+           "lx_score_topk")
+    return plan
+
+
+def lx_sparse_attn_plan(Q, K, keep, plan: Plan | None = None, ws=None, stream=None, with_mask=True) -> Plan:
+    lib = _abi.load()
+    B, H, L, D = Q.shape
+    _, _, _, wb = lx_plan_size(B, H, L, D, keep)
+    if plan is None:
+        plan = empty_plan(B, H, L, D, keep, Q.device, with_mask)
+    if ws is None:
+        ws = torch.empty(wb, dtype=torch.uint8, device=Q.device)
+    q, k, cp = bhld(Q), bhld(K), plan.c()
+    _check(lib.lx_sparse_attn_plan(ctypes.byref(q), ctypes.byref(k), float(keep), ctypes.byref(cp), _ptr(ws),
+                                   ws.numel(), _stream(stream)), "lx_sparse_attn_plan")
+    return plan
+
+
+def lx_quantize_qk(Q, K, out=None, stream=None):
+    lib = _abi.load()
+    B, H, L, D = Q.shape
+    nB = (L + LX_BLOCK - 1) // LX_BLOCK
+    if out is None:
+        dev = Q.device
+        out = (torch.empty((B, H, L, D), dtype=torch.int8, device=dev),
+               torch.empty((B, H, nB), dtype=torch.float32, device=dev),
+               torch.empty((B, H, L, D), dtype=torch.int8, device=dev),
+               torch.empty((B, H, nB), dtype=torch.float32, device=dev))
+    qc, qs, kc, ks = out
+    q, k = bhld(Q), bhld(K)
+    _check(lib.lx_quantize_qk(ctypes.byref(q), ctypes.byref(k), _ptr(qc), _ptr(qs), _ptr(kc), _ptr(ks),
+                              _stream(stream)), "lx_quantize_qk")
+    return out
+
+
+def lx_quantize_v(V, out=None, amax_ws=None, stream=None):
+    lib = _abi.load()
+    B, H, L, D = V.shape
+    if out is None:
+        out = (torch.empty((B, H, L, D), dtype=torch.uint8, device=V.device),
+               torch.empty((B, H, D), dtype=torch.float32, device=V.device))
+    if amax_ws is None:
+        amax_ws = torch.empty((B, H, D), dtype=torch.int32, device=V.device)
+    v = bhld(V)
+    _check(lib.lx_quantize_v(ctypes.byref(v), _ptr(out[0]), _ptr(out[1]), _ptr(amax_ws), _stream(stream)),
+           "lx_quantize_v")
+    return out
+
+
+def lx_attn_bf16(Q, K, V, plan: Plan, out=None, stream=None):
+    lib = _abi.load()
+    if out is None:
+        out = torch.empty_like(Q)
+    q, k, v, o, cp = bhld(Q), bhld(K), bhld(V), bhld(out), plan.c()
+    _check(lib.lx_attn_bf16(ctypes.byref(q), ctypes.byref(k), ctypes.byref(v), ctypes.byref(cp), ctypes.byref(o),
+                            _stream(stream)), "lx_attn_bf16")
+    return out
+
+
+def lx_attn_int8fp8(qc, qs, kc, ks, vc, vs, plan: Plan, out=None, stream=None):
+    lib = _abi.load()
+    if out is None:
+        out = torch.empty(qc.shape, dtype=torch.bfloat16, device=qc.device)
+    o, cp = bhld(out), plan.c()
+    _check(lib.lx_attn_int8fp8(_ptr(qc), _ptr(qs), _ptr(kc), _ptr(ks), _ptr(vc), _ptr(vs), ctypes.byref(cp),
+                               ctypes.byref(o), _stream(stream)), "lx_attn_int8fp8")
+    return out
+
+
+def lx_fwd_workspace_size(Q, mode) -> int:
+    lib = _abi.load()
+    n = ctypes.c_size_t()
+    q = bhld(Q)
+    _check(lib.lx_fwd_workspace_size(ctypes.byref(q), MODES[mode], ctypes.byref(n)), "lx_fwd_workspace_size")
+    return n.value
+
+
+def lx_sparse_attn_fwd(Q, K, V, plan: Plan, mode="int8fp8", out=None, ws=None, stream=None):
+    lib = _abi.load()
+    if out is None:
+        out = torch.empty_like(Q)
+    if ws is None:
+        n = lx_fwd_workspace_size(Q, mode)
+        ws = torch.empty(max(n, 256), dtype=torch.uint8, device=Q.device)
+    q, k, v, o, cp = bhld(Q), bhld(K), bhld(V), bhld(out), plan.c()
+    _check(lib.lx_sparse_attn_fwd(ctypes.byref(q), ctypes.byref(k), ctypes.byref(v), ctypes.byref(cp), MODES[mode],
+                                  ctypes.byref(o), _ptr(ws), ws.numel(), _stream(stream)), "lx_sparse_attn_fwd")
+    return out
+
+
+def lx_last_device_status(stream=None) -> int:
+    return _abi.load().lx_last_device_status(_stream(stream))
+
+
+def lx_debug_wait_timeout(limit_ns: int, stream=None):
+    _check(_abi.load().lx_debug_wait_timeout(int(limit_ns), _stream(stream)), "lx_debug_wait_timeout")
+
+
+def keep_count(nB: int, keep: float) -> int:
+    """k for a plan, from the library's own size query (nB blocks of 64)."""
+    return lx_plan_size(1, 1, nB * LX_BLOCK, 64, keep)[0]
+
+
+def effective_flops(B, H, L, D, keep) -> float:
+    """4 L^2 D H B * k/nB: the attention work on the kept tiles only."""
+    nB = math.ceil(L / LX_BLOCK)
+    k = keep_count(nB, keep)
+    return 4.0 * L * L * D * H * B * k / nB

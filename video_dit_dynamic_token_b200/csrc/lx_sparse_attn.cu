@@ -1,0 +1,382 @@
+// C-ABI host library: argument checks, TMA tensor maps, launches.
+// The whole library is this one translation unit (kernels come in as headers).
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+
+#include "lx_sparse_attn.h"
+#include "ptx.cuh"
+#include "planner.cuh"
+#include "quant.cuh"
+#include "attn.cuh"
+
+namespace {
+
+constexpr unsigned long long kWaitLimitNs = 2000000000ull;  // bound on every device-side wait
+constexpr int64_t kMaxPlannerNB = 2432;                       // score rows of 16 x nB fp32 in shared memory
+
+inline bool al16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+inline int64_t n_blocks(int64_t L) { return (L + LX_BLOCK - 1) / LX_BLOCK; }
+inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+inline int64_t keep_count(int64_t nB, double keep) {
+  int64_t k = (int64_t)std::ceil(keep * (double)nB - 1e-6);
+  return k < 1 ? 1 : (k > nB ? nB : k);
+}
+
+lx_status check_bhld(const lx_bhld* t) {
+  if (!t || !t->data) return LX_ERR_INVALID;
+  if (t->B < 1 || t->H < 1 || t->L < 1) return LX_ERR_INVALID;
+  if (t->D != 64 && t->D != 128) return LX_ERR_UNSUPPORTED;
+  if (t->sL < t->D || t->sH < 1 || t->sB < 1) return LX_ERR_INVALID;
+  if (t->L > (int64_t)1 << 30 || t->B * t->H > (int64_t)1 << 30) return LX_ERR_UNSUPPORTED;
+  if (!al16(t->data) || (t->sL * 2) % 16 || (t->sH * 2) % 16 || (t->sB * 2) % 16) return LX_ERR_ALIGN;
+  return LX_OK;
+}
+
+inline bool same_shape(const lx_bhld* a, const lx_bhld* b) {
+  return a->B == b->B && a->H == b->H && a->L == b->L && a->D == b->D;
+}
+
+inline lx::BhldView view(const lx_bhld* t) {
+  return lx::BhldView{reinterpret_cast<const __nv_bfloat16*>(t->data), t->sB, t->sH, t->sL};
+}
+
+lx_status check_plan(const lx_plan* p, const lx_bhld* shape) {
+  if (!p || !p->idx || !al16(p->idx)) return LX_ERR_INVALID;
+  const int64_t nB = n_blocks(shape->L);
+  if (p->B != shape->B || p->H != shape->H || p->L != shape->L || p->nB != nB || p->block != LX_BLOCK)
+    return LX_ERR_INVALID;
+  if (p->k < 1 || p->k > nB) return LX_ERR_INVALID;
+  return LX_OK;
+}
+
+inline lx_status launch_status() {
+  return cudaGetLastError() == cudaSuccess ? LX_OK : LX_ERR_CUDA;
+}
+
+// ---------------------------------------------------------------- TMA maps
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+// 4-D map over [B,H,L,D] (innermost first: D, L, H, B), strides in elements.
+bool make_map(CUtensorMap* m, const void* ptr, CUtensorMapDataType dt, int esz, int64_t B, int64_t H, int64_t L,
+              int64_t D, int64_t sB, int64_t sH, int64_t sL, int box_inner, int box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[4] = {(cuuint64_t)D, (cuuint64_t)L, (cuuint64_t)H, (cuuint64_t)B};
+  const cuuint64_t strides[3] = {(cuuint64_t)(sL * esz), (cuuint64_t)(sH * esz), (cuuint64_t)(sB * esz)};
+  const cuuint32_t box[4] = {(cuuint32_t)box_inner, (cuuint32_t)box_rows, 1, 1};
+  const cuuint32_t es[4] = {1, 1, 1, 1};
+  const int inner_bytes = box_inner * esz;
+  const CUtensorMapSwizzle sw = inner_bytes == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
+  return fn(m, dt, 4, const_cast<void*>(ptr), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// ---------------------------------------------------------------- launchers
+template <int D>
+lx_status launch_pool(const lx_bhld* Q, const lx_bhld* K, float* mq, float* mk, cudaStream_t s) {
+  const int64_t nB = n_blocks(Q->L);
+  const long long units = (long long)(Q->B * Q->H * nB);
+  dim3 grid((unsigned)((units + 7) / 8), 2);
+  lx::pool_means_kernel<D><<<grid, 256, 0, s>>>(view(Q), view(K), mq, mk, (int)Q->H, (int)Q->L, (int)nB, units);
+  return launch_status();
+}
+
+template <int D>
+lx_status launch_score(const float* mq, const float* mk, int64_t BH, int64_t nB, int64_t k, lx_plan* plan,
+                       cudaStream_t s) {
+  const int ldS = (int)((nB + 31) / 32 * 32);
+  const size_t smem = sizeof(float) * ((size_t)lx::kScoreRows * ldS + (size_t)lx::kKeyChunk * D + 8 * 256 +
+                                       2 * 8 * lx::kCandCap + 8 * (ldS / 32));
+  if (cudaFuncSetAttribute(lx::score_topk_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+      cudaSuccess)
+    return LX_ERR_CUDA;
+  dim3 grid((unsigned)((nB + lx::kScoreRows - 1) / lx::kScoreRows), (unsigned)BH);
+  lx::score_topk_kernel<D><<<grid, 256, smem, s>>>(mq, mk, (int)nB, (int)k, plan->idx, plan->mask, ldS);
+  return launch_status();
+}
+
+template <int D>
+lx_status launch_quant_qk(const lx_bhld* Q, const lx_bhld* K, int8_t* qc, float* qs, int8_t* kc, float* ks,
+                          cudaStream_t s) {
+  const int64_t nB = n_blocks(Q->L);
+  dim3 grid((unsigned)(Q->B * Q->H * nB), 2);
+  lx::quant_qk_kernel<D><<<grid, 128, 0, s>>>(view(Q), view(K), qc, kc, qs, ks, (int)Q->H, (int)Q->L, (int)nB);
+  return launch_status();
+}
+
+template <int D>
+lx_status launch_quant_v(const lx_bhld* V, uint8_t* vc, float* vs, uint32_t* amax, cudaStream_t s) {
+  const int64_t BH = V->B * V->H, nB = n_blocks(V->L);
+  const int nSpan = (int)((V->L + lx::kVSpan - 1) / lx::kVSpan);
+  if (cudaMemsetAsync(amax, 0, sizeof(uint32_t) * BH * D, s) != cudaSuccess) return LX_ERR_CUDA;
+  lx::v_absmax_kernel<D><<<(unsigned)(BH * nSpan), 128, 0, s>>>(view(V), amax, (int)V->H, (int)V->L, nSpan);
+  if (cudaGetLastError() != cudaSuccess) return LX_ERR_CUDA;
+  lx::v_quant_kernel<D><<<(unsigned)(BH * nB), 128, 0, s>>>(view(V), amax, vc, vs, (int)V->H, (int)V->L, (int)nB);
+  return launch_status();
+}
+
+template <int D, bool I8>
+lx_status launch_attn(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const lx_plan* plan,
+                      const lx_bhld* O, const float* qs, const float* ks, const float* vs, cudaStream_t s) {
+  using C = lx::AttnCfg<D, I8>;
+  const int64_t nB = plan->nB;
+  const int nW = (int)((nB + 31) / 32);
+  const size_t smem = 1024 + C::OFF_MASK + 2 * sizeof(uint32_t) * nW;
+  if (smem > 227 * 1024) return LX_ERR_UNSUPPORTED;
+  if (cudaFuncSetAttribute(lx::sparse_attn_kernel<D, I8>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+      cudaSuccess)
+    return LX_ERR_CUDA;
+  lx::AttnParams p;
+  p.idx = plan->idx;
+  p.k = (int)plan->k;
+  p.nB = (int)nB;
+  p.L = (int)plan->L;
+  p.H = (int)plan->H;
+  p.o = reinterpret_cast<__nv_bfloat16*>(O->data);
+  p.osB = O->sB;
+  p.osH = O->sH;
+  p.osL = O->sL;
+  p.sq = qs;
+  p.sk = ks;
+  p.sv = vs;
+  p.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)D));
+  p.limit_ns = kWaitLimitNs;
+  dim3 grid((unsigned)((nB + 1) / 2), (unsigned)(plan->B * plan->H));
+  lx::sparse_attn_kernel<D, I8><<<grid, 192, smem, s>>>(mq, mk, mv, p);
+  return launch_status();
+}
+
+template <int D>
+lx_status attn_bf16_impl(const lx_bhld* Q, const lx_bhld* K, const lx_bhld* V, const lx_plan* plan, const lx_bhld* O,
+                         cudaStream_t s) {
+  CUtensorMap mq, mk, mv;
+  const auto dt = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  if (!make_map(&mq, Q->data, dt, 2, Q->B, Q->H, Q->L, D, Q->sB, Q->sH, Q->sL, 64, 128) ||
+      !make_map(&mk, K->data, dt, 2, K->B, K->H, K->L, D, K->sB, K->sH, K->sL, 64, 64) ||
+      !make_map(&mv, V->data, dt, 2, V->B, V->H, V->L, D, V->sB, V->sH, V->sL, 64, 64))
+    return LX_ERR_CUDA;
+  return launch_attn<D, false>(mq, mk, mv, plan, O, nullptr, nullptr, nullptr, s);
+}
+
+template <int D>
+lx_status attn_i8_impl(const int8_t* qc, const float* qs, const int8_t* kc, const float* ks, const uint8_t* vc,
+                       const float* vs, const lx_plan* plan, const lx_bhld* O, cudaStream_t s) {
+  CUtensorMap mq, mk, mv;
+  const int64_t B = O->B, H = O->H, L = O->L;
+  const int64_t sL = D, sH = L * D, sB = H * L * D;
+  const auto dt = CU_TENSOR_MAP_DATA_TYPE_UINT8;
+  if (!make_map(&mq, qc, dt, 1, B, H, L, D, sB, sH, sL, D, 128) ||
+      !make_map(&mk, kc, dt, 1, B, H, L, D, sB, sH, sL, D, 64) ||
+      !make_map(&mv, vc, dt, 1, B, H, L, D, sB, sH, sL, D, 64))
+    return LX_ERR_CUDA;
+  return launch_attn<D, true>(mq, mk, mv, plan, O, qs, ks, vs, s);
+}
+
+struct FwdWs {
+  size_t qc, kc, vc, qs, ks, vs, amax, total;
+};
+FwdWs fwd_layout(const lx_bhld* Q) {
+  FwdWs w;
+  const size_t codes = (size_t)(Q->B * Q->H * Q->L * Q->D);
+  const size_t bsc = sizeof(float) * (size_t)(Q->B * Q->H * n_blocks(Q->L));
+  const size_t csc = sizeof(float) * (size_t)(Q->B * Q->H * Q->D);
+  w.qc = 0;
+  w.kc = w.qc + align256(codes);
+  w.vc = w.kc + align256(codes);
+  w.qs = w.vc + align256(codes);
+  w.ks = w.qs + align256(bsc);
+  w.vs = w.ks + align256(bsc);
+  w.amax = w.vs + align256(csc);
+  w.total = w.amax + align256(csc);
+  return w;
+}
+
+}  // namespace
+
+// ====================================================================== C ABI
+extern "C" {
+
+const char* lx_status_string(lx_status st) {
+  switch (st) {
+    case LX_OK: return "ok";
+    case LX_ERR_INVALID: return "invalid argument";
+    case LX_ERR_UNSUPPORTED: return "unsupported shape";
+    case LX_ERR_ALIGN: return "pointer or stride not 16-byte aligned";
+    case LX_ERR_WORKSPACE: return "workspace missing or too small";
+    case LX_ERR_CUDA: return "CUDA error";
+    case LX_ERR_TIMEOUT: return "device wait timed out";
+    case LX_ERR_PLAN: return "malformed plan or non-finite scores";
+  }
+  return "unknown status";
+}
+
+lx_status lx_plan_size(int64_t B, int64_t H, int64_t L, int64_t D, double keep, int64_t* k, size_t* idx_bytes,
+                       size_t* mask_bytes, size_t* ws_bytes) {
+  if (B < 1 || H < 1 || L < 1 || !(keep > 0.0 && keep <= 1.0)) return LX_ERR_INVALID;
+  if (D != 64 && D != 128) return LX_ERR_UNSUPPORTED;
+  const int64_t nB = n_blocks(L), kk = keep_count(nB, keep);
+  if (k) *k = kk;
+  if (idx_bytes) *idx_bytes = sizeof(int32_t) * (size_t)(B * H * nB * kk);
+  if (mask_bytes) *mask_bytes = sizeof(uint32_t) * (size_t)(B * H * nB * ((nB + 31) / 32));
+  if (ws_bytes) *ws_bytes = 2 * align256(sizeof(float) * (size_t)(B * H * nB * D));
+  return LX_OK;
+}
+
+lx_status lx_pool_means(const lx_bhld* Q, const lx_bhld* K, float* mq, float* mk, cudaStream_t stream) {
+  lx_status st;
+  if ((st = check_bhld(Q)) != LX_OK || (st = check_bhld(K)) != LX_OK) return st;
+  if (!same_shape(Q, K) || !mq || !mk) return LX_ERR_INVALID;
+  if (!al16(mq) || !al16(mk)) return LX_ERR_ALIGN;
+  return Q->D == 128 ? launch_pool<128>(Q, K, mq, mk, stream) : launch_pool<64>(Q, K, mq, mk, stream);
+}
+
+lx_status lx_score_topk(const float* mq, const float* mk, int64_t B, int64_t H, int64_t L, int64_t D, double keep,
+                        lx_plan* plan, cudaStream_t stream) {
+  int64_t k = 0;
+  lx_status st = lx_plan_size(B, H, L, D, keep, &k, nullptr, nullptr, nullptr);
+  if (st != LX_OK) return st;
+  if (!mq || !mk || !plan || !plan->idx) return LX_ERR_INVALID;
+  if (!al16(mq) || !al16(mk) || !al16(plan->idx) || (plan->mask && !al16(plan->mask))) return LX_ERR_ALIGN;
+  const int64_t nB = n_blocks(L);
+  if (nB > kMaxPlannerNB) return LX_ERR_UNSUPPORTED;
+  plan->B = B;
+  plan->H = H;
+  plan->L = L;
+  plan->nB = nB;
+  plan->k = k;
+  plan->block = LX_BLOCK;
+  return D == 128 ? launch_score<128>(mq, mk, B * H, nB, k, plan, stream)
+                  : launch_score<64>(mq, mk, B * H, nB, k, plan, stream);
+}
+
+lx_status lx_sparse_attn_plan(const lx_bhld* Q, const lx_bhld* K, double keep, lx_plan* plan, void* ws,
+                              size_t ws_bytes, cudaStream_t stream) {
+  lx_status st;
+  if ((st = check_bhld(Q)) != LX_OK || (st = check_bhld(K)) != LX_OK) return st;
+  if (!same_shape(Q, K) || !plan) return LX_ERR_INVALID;
+  size_t need = 0;
+  if ((st = lx_plan_size(Q->B, Q->H, Q->L, Q->D, keep, nullptr, nullptr, nullptr, &need)) != LX_OK) return st;
+  if (!ws || ws_bytes < need) return LX_ERR_WORKSPACE;
+  if (!al16(ws)) return LX_ERR_ALIGN;
+  if (n_blocks(Q->L) > kMaxPlannerNB) return LX_ERR_UNSUPPORTED;
+  float* mq = reinterpret_cast<float*>(ws);
+  float* mk = reinterpret_cast<float*>(reinterpret_cast<char*>(ws) + need / 2);
+  if ((st = lx_pool_means(Q, K, mq, mk, stream)) != LX_OK) return st;
+  return lx_score_topk(mq, mk, Q->B, Q->H, Q->L, Q->D, keep, plan, stream);
+}
+
+lx_status lx_quantize_qk(const lx_bhld* Q, const lx_bhld* K, int8_t* qc, float* qs, int8_t* kc, float* ks,
+                         cudaStream_t stream) {
+  lx_status st;
+  if ((st = check_bhld(Q)) != LX_OK || (st = check_bhld(K)) != LX_OK) return st;
+  if (!same_shape(Q, K) || !qc || !qs || !kc || !ks) return LX_ERR_INVALID;
+  if (!al16(qc) || !al16(kc) || !al16(qs) || !al16(ks)) return LX_ERR_ALIGN;
+  return Q->D == 128 ? launch_quant_qk<128>(Q, K, qc, qs, kc, ks, stream)
+                     : launch_quant_qk<64>(Q, K, qc, qs, kc, ks, stream);
+}
+
+lx_status lx_quantize_v(const lx_bhld* V, uint8_t* vc, float* vs, uint32_t* amax_ws, cudaStream_t stream) {
+  lx_status st;
+  if ((st = check_bhld(V)) != LX_OK) return st;
+  if (!vc || !vs || !amax_ws) return LX_ERR_INVALID;
+  if (!al16(vc) || !al16(vs) || !al16(amax_ws)) return LX_ERR_ALIGN;
+  return V->D == 128 ? launch_quant_v<128>(V, vc, vs, amax_ws, stream)
+                     : launch_quant_v<64>(V, vc, vs, amax_ws, stream);
+}
+
+lx_status lx_attn_bf16(const lx_bhld* Q, const lx_bhld* K, const lx_bhld* V, const lx_plan* plan, const lx_bhld* O,
+                       cudaStream_t stream) {
+  lx_status st;
+  if ((st = check_bhld(Q)) != LX_OK || (st = check_bhld(K)) != LX_OK || (st = check_bhld(V)) != LX_OK ||
+      (st = check_bhld(O)) != LX_OK)
+    return st;
+  if (!same_shape(Q, K) || !same_shape(Q, V) || !same_shape(Q, O)) return LX_ERR_INVALID;
+  if ((st = check_plan(plan, Q)) != LX_OK) return st;
+  return Q->D == 128 ? attn_bf16_impl<128>(Q, K, V, plan, O, stream) : attn_bf16_impl<64>(Q, K, V, plan, O, stream);
+}
+
+lx_status lx_attn_int8fp8(const int8_t* qc, const float* qs, const int8_t* kc, const float* ks, const uint8_t* vc,
+                          const float* vs, const lx_plan* plan, const lx_bhld* O, cudaStream_t stream) {
+  lx_status st;
+  if ((st = check_bhld(O)) != LX_OK) return st;
+  if (!qc || !qs || !kc || !ks || !vc || !vs) return LX_ERR_INVALID;
+  if (!al16(qc) || !al16(kc) || !al16(vc) || !al16(qs) || !al16(ks) || !al16(vs)) return LX_ERR_ALIGN;
+  if ((st = check_plan(plan, O)) != LX_OK) return st;
+  return O->D == 128 ? attn_i8_impl<128>(qc, qs, kc, ks, vc, vs, plan, O, stream)
+                     : attn_i8_impl<64>(qc, qs, kc, ks, vc, vs, plan, O, stream);
+}
+
+lx_status lx_fwd_workspace_size(const lx_bhld* Q, lx_mode mode, size_t* bytes) {
+  if (!Q || !bytes) return LX_ERR_INVALID;
+  if (Q->B < 1 || Q->H < 1 || Q->L < 1) return LX_ERR_INVALID;
+  if (Q->D != 64 && Q->D != 128) return LX_ERR_UNSUPPORTED;
+  if (mode == LX_MODE_BF16) {
+    *bytes = 0;
+    return LX_OK;
+  }
+  if (mode != LX_MODE_INT8FP8) return LX_ERR_INVALID;
+  *bytes = fwd_layout(Q).total;
+  return LX_OK;
+}
+
+lx_status lx_sparse_attn_fwd(const lx_bhld* Q, const lx_bhld* K, const lx_bhld* V, const lx_plan* plan, lx_mode mode,
+                             const lx_bhld* O, void* ws, size_t ws_bytes, cudaStream_t stream) {
+  if (mode == LX_MODE_BF16) return lx_attn_bf16(Q, K, V, plan, O, stream);
+  if (mode != LX_MODE_INT8FP8) return LX_ERR_INVALID;
+  lx_status st;
+  if ((st = check_bhld(Q)) != LX_OK || (st = check_bhld(K)) != LX_OK || (st = check_bhld(V)) != LX_OK ||
+      (st = check_bhld(O)) != LX_OK)
+    return st;
+  if (!same_shape(Q, K) || !same_shape(Q, V) || !same_shape(Q, O)) return LX_ERR_INVALID;
+  if ((st = check_plan(plan, Q)) != LX_OK) return st;
+  const FwdWs w = fwd_layout(Q);
+  if (!ws || ws_bytes < w.total) return LX_ERR_WORKSPACE;
+  if ((reinterpret_cast<uintptr_t>(ws) & 255u) != 0) return LX_ERR_ALIGN;
+  char* base = reinterpret_cast<char*>(ws);
+  int8_t* qc = reinterpret_cast<int8_t*>(base + w.qc);
+  int8_t* kc = reinterpret_cast<int8_t*>(base + w.kc);
+  uint8_t* vc = reinterpret_cast<uint8_t*>(base + w.vc);
+  float* qs = reinterpret_cast<float*>(base + w.qs);
+  float* ks = reinterpret_cast<float*>(base + w.ks);
+  float* vs = reinterpret_cast<float*>(base + w.vs);
+  uint32_t* amax = reinterpret_cast<uint32_t*>(base + w.amax);
+  if ((st = lx_quantize_qk(Q, K, qc, qs, kc, ks, stream)) != LX_OK) return st;
+  if ((st = lx_quantize_v(V, vc, vs, amax, stream)) != LX_OK) return st;
+  return lx_attn_int8fp8(qc, qs, kc, ks, vc, vs, plan, O, stream);
+}
+
+lx_status lx_last_device_status(cudaStream_t stream) {
+  if (cudaStreamSynchronize(stream) != cudaSuccess) return LX_ERR_CUDA;
+  int v = 0;
+  if (cudaMemcpyFromSymbol(&v, lx::g_device_status, sizeof(int)) != cudaSuccess) return LX_ERR_CUDA;
+  const int zero = 0;
+  if (v != 0 && cudaMemcpyToSymbol(lx::g_device_status, &zero, sizeof(int)) != cudaSuccess) return LX_ERR_CUDA;
+  if (v == LX_ERR_TIMEOUT || v == LX_ERR_PLAN) return (lx_status)v;
+  return v == 0 ? LX_OK : LX_ERR_CUDA;
+}
+
+lx_status lx_debug_wait_timeout(uint64_t limit_ns, cudaStream_t stream) {
+  if (limit_ns == 0 || limit_ns > 10000000000ull) return LX_ERR_INVALID;
+  lx::wait_timeout_probe_kernel<<<1, 32, 0, stream>>>((unsigned long long)limit_ns);
+  return launch_status();
+}
+
+}  // extern "C"

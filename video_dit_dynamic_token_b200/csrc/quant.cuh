@@ -1,0 +1,172 @@
+// Quantisers (step a3): Q and K to INT8 with one symmetric scale per
+// (b, h, 64-token block); V to FP8 E4M3 with one scale per (b, h, channel).
+//
+// "600倍加速，720p视频实时生成！单卡也能带的动14B模型", §高效推理算子: the sparse
+// attention runs with Q/K in INT8 and V in FP8.  The scale granularity is this
+// library's reading: absmax/127 per block for Q/K, absmax/448 per channel for V,
+// codes rint(x*(127/a)) clamped to +-127 and E4M3_rn_satfinite(v*(448/a)); both
+// code decisions are taken in fp32 with correctly rounded divide and multiply.
+#pragma once
+#include <cuda_bf16.h>
+#include <cstdint>
+#include "planner.cuh"
+
+namespace lx {
+
+__device__ __forceinline__ float bf16lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+
+__device__ __forceinline__ uint32_t pack_i8x4(int a, int b, int c, int d) {
+  return (uint32_t)(a & 0xFF) | ((uint32_t)(b & 0xFF) << 8) | ((uint32_t)(c & 0xFF) << 16) | ((uint32_t)(d & 0xFF) << 24);
+}
+
+__device__ __forceinline__ int quant_i8(float x, float inv) {
+  const int q = __float2int_rn(__fmul_rn(x, inv));  // round half to even
+  return max(-127, min(127, q));
+}
+
+// Two fp32 values to two E4M3 codes (lo in bits 0..7), round to nearest even, saturating.
+__device__ __forceinline__ uint32_t e4m3x2(float lo, float hi) {
+  uint16_t r;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
+  return (uint32_t)r;
+}
+
+// ---------------------------------------------------------------------------
+// Q/K: one 128-thread CTA per (tensor, b*h, block).  Thread t covers row t/2,
+// half (t&1) of the D channels (D/2 values = D/16 16-byte chunks).
+template <int D>
+__global__ void __launch_bounds__(128) quant_qk_kernel(BhldView q, BhldView k, int8_t* __restrict__ qc,
+                                                      int8_t* __restrict__ kc, float* __restrict__ qs,
+                                                      float* __restrict__ ks, int H, int L, int nB) {
+  constexpr int NCH = D / 16;  // 16-byte input chunks per thread
+  const BhldView X = blockIdx.y == 0 ? q : k;
+  int8_t* __restrict__ C = blockIdx.y == 0 ? qc : kc;
+  float* __restrict__ S = blockIdx.y == 0 ? qs : ks;
+  const long long unit = blockIdx.x;
+  const long long bh = unit / nB;
+  const int blk = (int)(unit - bh * nB);
+  const long long b = bh / H, h = bh - b * H;
+  const int t0 = blk * kBlock;
+  const int cnt = min(kBlock, L - t0);
+  const int row = threadIdx.x >> 1, col0 = (threadIdx.x & 1) * (D / 2);
+  uint4 v[NCH];
+  const __nv_bfloat16* src = X.p + b * X.sB + h * X.sH + (long long)(t0 + row) * X.sL + col0;
+#pragma unroll
+  for (int i = 0; i < NCH; ++i) v[i] = row < cnt ? ld_stream_v4(src + 8 * i) : make_uint4(0, 0, 0, 0);
+  float a = 0.f;
+#pragma unroll
+  for (int i = 0; i < NCH; ++i) {
+    const uint32_t w[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) a = fmaxf(a, fmaxf(fabsf(bf16lo(w[e])), fabsf(bf16hi(w[e]))));
+  }
+#pragma unroll
+  for (int off = 16; off; off >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, off));
+  __shared__ float red[4];
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = a;
+  __syncthreads();
+  a = fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3]));
+  const float inv = a > 0.f ? __fdiv_rn(127.0f, a) : 0.f;
+  if (row < cnt) {
+    int8_t* dst = C + (bh * L + t0 + row) * D + col0;
+#pragma unroll
+    for (int i = 0; i < NCH; i += 2) {
+      uint32_t o[4];
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh) {
+        const uint32_t w[4] = {v[i + hh].x, v[i + hh].y, v[i + hh].z, v[i + hh].w};
+        o[2 * hh] = pack_i8x4(quant_i8(bf16lo(w[0]), inv), quant_i8(bf16hi(w[0]), inv), quant_i8(bf16lo(w[1]), inv),
+                              quant_i8(bf16hi(w[1]), inv));
+        o[2 * hh + 1] = pack_i8x4(quant_i8(bf16lo(w[2]), inv), quant_i8(bf16hi(w[2]), inv),
+                                  quant_i8(bf16lo(w[3]), inv), quant_i8(bf16hi(w[3]), inv));
+      }
+      *reinterpret_cast<uint4*>(dst + 8 * i) = make_uint4(o[0], o[1], o[2], o[3]);
+    }
+  }
+  if (threadIdx.x == 0) S[bh * nB + blk] = a > 0.f ? __fdiv_rn(a, 127.0f) : 1.0f;
+}
+
+// ---------------------------------------------------------------------------
+// V, pass 1: per-channel absmax.  One 128-thread CTA per (b*h, 512-token span);
+// lanes cover 16-byte channel chunks; the CTA folds its rows in shared memory
+// and merges into the (zero-initialised) per-channel maxima with atomicMax on
+// the bit patterns (non-negative floats order like unsigned ints).
+constexpr int kVSpan = 512;
+template <int D>
+__global__ void __launch_bounds__(128) v_absmax_kernel(BhldView v, uint32_t* __restrict__ amax, int H, int L,
+                                                      int nSpan) {
+  constexpr int CH = D / 8;        // chunks per row
+  constexpr int RPP = 128 / CH;    // rows per pass
+  const long long bh = blockIdx.x / nSpan;
+  const int span = (int)(blockIdx.x - bh * nSpan);
+  const long long b = bh / H, h = bh - b * H;
+  const int c = threadIdx.x % CH, r0 = threadIdx.x / CH;
+  const int t_begin = span * kVSpan, t_end = min(L, t_begin + kVSpan);
+  float m[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+  const __nv_bfloat16* base = v.p + b * v.sB + h * v.sH + c * 8;
+  for (int t = t_begin + r0; t < t_end; t += RPP) {
+    const uint4 x = ld_stream_v4(base + (long long)t * v.sL);
+    const uint32_t w[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      m[2 * e] = fmaxf(m[2 * e], fabsf(bf16lo(w[e])));
+      m[2 * e + 1] = fmaxf(m[2 * e + 1], fabsf(bf16hi(w[e])));
+    }
+  }
+  __shared__ float red[128][9];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) red[threadIdx.x][e] = m[e];
+  __syncthreads();
+  if (threadIdx.x < D) {
+    const int ch = threadIdx.x / 8, e = threadIdx.x % 8;
+    float mm = 0.f;
+    for (int r = 0; r < RPP; ++r) mm = fmaxf(mm, red[r * CH + ch][e]);
+    atomicMax(amax + bh * D + threadIdx.x, __float_as_uint(mm));
+  }
+}
+
+// V, pass 2: codes.  One 128-thread CTA per (b*h, 64-token block); thread t
+// covers row t/2 and half of the channels, like quant_qk_kernel.  The CTA of
+// block 0 also writes the per-channel scales.
+template <int D>
+__global__ void __launch_bounds__(128) v_quant_kernel(BhldView v, const uint32_t* __restrict__ amax,
+                                                     uint8_t* __restrict__ vc, float* __restrict__ vs, int H, int L,
+                                                     int nB) {
+  constexpr int NCH = D / 16;
+  const long long bh = blockIdx.x / nB;
+  const int blk = (int)(blockIdx.x - bh * nB);
+  const long long b = bh / H, h = bh - b * H;
+  const int t0 = blk * kBlock;
+  const int cnt = min(kBlock, L - t0);
+  __shared__ float inv_s[D];
+  for (int ch = threadIdx.x; ch < D; ch += blockDim.x) {
+    const float a = __uint_as_float(amax[bh * D + ch]);
+    inv_s[ch] = a > 0.f ? __fdiv_rn(448.0f, a) : 0.f;
+    if (blk == 0) vs[bh * D + ch] = a > 0.f ? __fdiv_rn(a, 448.0f) : 1.0f;
+  }
+  __syncthreads();
+  const int row = threadIdx.x >> 1, col0 = (threadIdx.x & 1) * (D / 2);
+  if (row >= cnt) return;
+  const __nv_bfloat16* src = v.p + b * v.sB + h * v.sH + (long long)(t0 + row) * v.sL + col0;
+  uint8_t* dst = vc + (bh * L + t0 + row) * D + col0;
+#pragma unroll
+  for (int i = 0; i < NCH; i += 2) {
+    uint32_t o[4];
+#pragma unroll
+    for (int hh = 0; hh < 2; ++hh) {
+      const uint4 x = ld_stream_v4(src + 8 * (i + hh));
+      const uint32_t w[4] = {x.x, x.y, x.z, x.w};
+      const float* iv = inv_s + col0 + 8 * (i + hh);
+      uint32_t p[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e)
+        p[e] = e4m3x2(__fmul_rn(bf16lo(w[e]), iv[2 * e]), __fmul_rn(bf16hi(w[e]), iv[2 * e + 1]));
+      o[2 * hh] = p[0] | (p[1] << 16);
+      o[2 * hh + 1] = p[2] | (p[3] << 16);
+    }
+    *reinterpret_cast<uint4*>(dst + 8 * i) = make_uint4(o[0], o[1], o[2], o[3]);
+  }
+}
+
+}  // namespace lx
