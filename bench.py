@@ -102,7 +102,7 @@ def run_ours(args, rank, world, local_rank):
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
     w = synth.WORKLOADS[WORKLOAD]
-    B, H, d, L, keep = w.B, w.H, w.d, w.L, w.keep
+    B, H, d, L, keep = w.B, args.heads or w.H, w.d, w.L, w.keep
     nB = math.ceil(L / 64)
     Q, K, V = synth.make_qkv(B, H, d, w.grid, seed=rank, device=dev)
     k, _, _, plan_ws_bytes = lx.lx_plan_size(B, H, L, d, keep)
@@ -316,6 +316,7 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--heads", type=int, default=0, help="fewer heads: a smaller case for profiling only")
     args = ap.parse_args()
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -334,7 +335,7 @@ def main():
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=__import__("torch").device("cuda", local_rank))
     cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and not args.heads:
         cpu = cpu_oracle_sample()
     out = run_ours(args, rank, world, local_rank)
     if world > 1:

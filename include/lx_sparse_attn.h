@@ -94,7 +94,7 @@ lx_status lx_pool_means(const lx_bhld* Q, const lx_bhld* K, float* mq, float* mk
  * plan->idx (and plan->mask when not NULL): per query block the k key blocks
  * with the largest mean(Q_i).mean(K_j)/sqrt(D), ties to the lower index,
  * ascending.  plan->idx/mask must be set by the caller; the call fills
- * plan->B, H, L, nB, k and block.  nB must not exceed 2432 (L <= 155648). */
+ * plan->B, H, L, nB, k and block.  nB must not exceed 2176 (L <= 139264). */
 lx_status lx_score_topk(const float* mq, const float* mk, int64_t B, int64_t H, int64_t L, int64_t D, double keep,
                         lx_plan* plan, cudaStream_t stream);
 

@@ -93,8 +93,8 @@ def test_host_argument_errors_before_launch(lib):
     assert lib.lx_sparse_attn_plan(ctypes.byref(q), ctypes.byref(q), 0.25, ctypes.byref(plan), 0x50000, 16, s) \
         == _abi.LX_ERR_WORKSPACE
     # planner beyond the selection kernel's row limit
-    huge = _view(L=64 * 2433, H=1)
-    _, _, _, _, wb = _plan_size(lib, 1, 1, 64 * 2433, 128, 0.1)
+    huge = _view(L=64 * 2177, H=1)
+    _, _, _, _, wb = _plan_size(lib, 1, 1, 64 * 2177, 128, 0.1)
     assert lib.lx_sparse_attn_plan(ctypes.byref(huge), ctypes.byref(huge), 0.1, ctypes.byref(plan), 0x50000, wb, s) \
         == _abi.LX_ERR_UNSUPPORTED
 

@@ -38,18 +38,16 @@ struct AttnCfg {
   static constexpr int NATOM = ROWB / ATOM;               // atom columns per row
   static constexpr int Q_BYTES = 128 * ROWB;
   static constexpr int KV_BYTES = 64 * ROWB;              // one K (or V) block
-  static constexpr int P_ROWB = 64 * ESZ;                 // P row: 64 keys
-  static constexpr int P_BYTES = 128 * P_ROWB;
-  static constexpr int NSTAGE = I8 ? 4 : 3;
+  static constexpr int NSTAGE = I8 ? 5 : 3;   // INT8: two CTAs fit one SM
   static constexpr uint32_t SW_QKV = ATOM == 128 ? SW_128B : SW_64B;
-  static constexpr uint32_t SW_P = P_ROWB == 128 ? SW_128B : SW_64B;
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_K = OFF_Q + Q_BYTES;
   static constexpr int OFF_V = OFF_K + NSTAGE * KV_BYTES;
-  static constexpr int OFF_P = OFF_V + NSTAGE * KV_BYTES;
-  static constexpr int OFF_MASK = OFF_P + 2 * P_BYTES;    // two bitmask rows follow
-  static constexpr int S_COL = 0;                         // TMEM: S buffers at cols 0 and 64
-  static constexpr int O_COL = 128;                       // TMEM: O accumulator
+  static constexpr int OFF_MASK = OFF_V + NSTAGE * KV_BYTES;  // two bitmask rows follow
+  static constexpr int P_COLS = 64 * ESZ / 4;             // P of one 64-key block: 16 (E4M3) or 32 (bf16) cols
+  static constexpr int S_COL = 0;                         // TMEM: S tile, cols [0, 64)
+  static constexpr int P_COL = 64;                        // TMEM: two P buffers, P_COLS each
+  static constexpr int O_COL = 128;                       // TMEM: O accumulator, D cols
   static constexpr uint32_t TMEM_COLS = 256;
   static constexpr uint32_t IDESC_S =
       instr_desc(I8 ? IDESC_DS32 : IDESC_DF32, I8 ? IDESC_S8 : IDESC_BF16, I8 ? IDESC_S8 : IDESC_BF16, 0, 0, 128, 64);
@@ -101,15 +99,22 @@ __device__ __forceinline__ float ex2f(float x) {
   return y;
 }
 
+// 12582912 = 1.5 * 2^23: an int32 s with |s| < 2^22 added to this float's bit
+// pattern gives the float 12582912 + s exactly.  The INT8 score accumulator is
+// started at this pattern, so the s32 QK^T result reads directly as a float.
+constexpr uint32_t kMagicBits = 0x4B400000u;
+constexpr float kMagic = 12582912.0f;
+constexpr float kLog2_448 = 8.807354922057604f;
+
 template <int D, bool I8>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(192, I8 ? 2 : 1)
     sparse_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                        const __grid_constant__ CUtensorMap tmV, const AttnParams prm) {
   using C = AttnCfg<D, I8>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  __shared__ uint64_t bar_q, bar_full[C::NSTAGE], bar_empty[C::NSTAGE], bar_sfull[2], bar_sfree[2], bar_pfull[2],
-      bar_odone, bar_drain;
+  __shared__ uint64_t bar_q, bar_full[C::NSTAGE], bar_empty[C::NSTAGE], bar_sfull, bar_sfree, bar_pfull[2], bar_odone,
+      bar_drain;
   __shared__ uint32_t tmem_slot;
   __shared__ volatile int abort_flag;
   __shared__ int n_union;
@@ -132,11 +137,9 @@ __global__ void __launch_bounds__(192, 1)
       mbar_init(&bar_full[s], 1);
       mbar_init(&bar_empty[s], 1);
     }
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(&bar_sfull[i], 1);
-      mbar_init(&bar_sfree[i], 128);
-      mbar_init(&bar_pfull[i], 128);
-    }
+    mbar_init(&bar_sfull, 1);
+    mbar_init(&bar_sfree, 128);
+    for (int i = 0; i < 2; ++i) mbar_init(&bar_pfull[i], 128);
     mbar_init(&bar_odone, 1);
     mbar_init(&bar_drain, 1);
     abort_flag = 0;
@@ -190,7 +193,7 @@ __global__ void __launch_bounds__(192, 1)
         tma_load_4d(sm + C::OFF_Q + a * 128 * C::ATOM, &tmQ, &bar_q, a * C::ATOM / C::ESZ, qb0 * kBlock, h_idx, b_idx);
       UnionWalk uw;
       uw.init(m0, m1, nW);
-      int j, fl, c = 0, issued = 0;
+      int j, fl, c = 0;
       while (uw.next(j, fl)) {
         const int s = c % C::NSTAGE;
         if (c >= C::NSTAGE && !mbar_wait(&bar_empty[s], ((c / C::NSTAGE) - 1) & 1, &abort_flag, prm.limit_ns)) {
@@ -206,11 +209,10 @@ __global__ void __launch_bounds__(192, 1)
                       j * kBlock, h_idx, b_idx);
         }
         ++c;
-        issued = c;
       }
       // drain: every issued load lands before the CTA may exit
       mbar_wait(&bar_q, 0, &never_abort, prm.limit_ns);
-      for (int cc = issued - C::NSTAGE < 0 ? 0 : issued - C::NSTAGE; cc < issued; ++cc)
+      for (int cc = c - C::NSTAGE < 0 ? 0 : c - C::NSTAGE; cc < c; ++cc)
         mbar_wait(&bar_full[cc % C::NSTAGE], (cc / C::NSTAGE) & 1, &never_abort, prm.limit_ns);
     }
   } else if (warp == 1) {
@@ -220,9 +222,9 @@ __global__ void __launch_bounds__(192, 1)
       tc_fence_after();
       for (int c = 0; ok && c <= n; ++c) {
         if (c < n) {
-          const int s = c % C::NSTAGE, bsel = c & 1;
-          ok = mbar_wait(&bar_full[s], (c / C::NSTAGE) & 1, &abort_flag, prm.limit_ns);
-          if (ok && c >= 2) ok = mbar_wait(&bar_sfree[bsel], ((c >> 1) - 1) & 1, &abort_flag, prm.limit_ns);
+          const int s = c % C::NSTAGE;
+          ok = mbar_wait(&bar_full[s], (c / C::NSTAGE) & 1, &abort_flag, prm.limit_ns) &&
+               mbar_wait(&bar_sfree, c & 1, &abort_flag, prm.limit_ns);
           if (!ok) break;
           tc_fence_after();
           const uint32_t sK = smem_u32(sm + C::OFF_K + s * C::KV_BYTES);
@@ -231,22 +233,22 @@ __global__ void __launch_bounds__(192, 1)
             const int a = (kk * 32) / C::ATOM, off = (kk * 32) % C::ATOM;
             const uint64_t ad = smem_desc(sQ + a * 128 * C::ATOM + off, 16, 8 * C::ATOM, C::SW_QKV);
             const uint64_t bd = smem_desc(sK + a * 64 * C::ATOM + off, 16, 8 * C::ATOM, C::SW_QKV);
-            mma_ss<I8 ? KIND_I8 : KIND_F16>(tbase + C::S_COL + bsel * 64, ad, bd, C::IDESC_S, kk > 0);
+            // INT8: accumulate onto the magic-number start the softmax warps wrote
+            mma_ss<I8 ? KIND_I8 : KIND_F16>(tbase + C::S_COL, ad, bd, C::IDESC_S, (I8 || kk > 0) ? 1u : 0u);
           }
-          mma_commit(&bar_sfull[bsel]);
+          mma_commit(&bar_sfull);
         }
         if (c >= 1) {
           const int cp = c - 1, s = cp % C::NSTAGE, pb = cp & 1;
           ok = mbar_wait(&bar_pfull[pb], (cp >> 1) & 1, &abort_flag, prm.limit_ns);
           if (!ok) break;
           tc_fence_after();
-          const uint32_t sP = smem_u32(sm + C::OFF_P + pb * C::P_BYTES);
           const uint32_t sV = smem_u32(sm + C::OFF_V + s * C::KV_BYTES);
 #pragma unroll
           for (int kk = 0; kk < 64 / C::KEYS_PER_MMA; ++kk) {
-            const uint64_t ad = smem_desc(sP + kk * 32, 16, 8 * C::P_ROWB, C::SW_P);
             const uint64_t bd = smem_desc(sV + kk * C::KEYS_PER_MMA * C::ATOM, 64 * C::ATOM, 8 * C::ATOM, C::SW_QKV);
-            mma_ss<I8 ? KIND_F8F6F4 : KIND_F16>(tbase + C::O_COL, ad, bd, C::IDESC_PV, (cp > 0 || kk > 0) ? 1u : 0u);
+            mma_ts<I8 ? KIND_F8F6F4 : KIND_F16>(tbase + C::O_COL, tbase + C::P_COL + pb * C::P_COLS + kk * 8, bd,
+                                                C::IDESC_PV, (cp > 0 || kk > 0) ? 1u : 0u);
           }
           mma_commit(&bar_odone);
           mma_commit(&bar_empty[s]);
@@ -268,8 +270,20 @@ __global__ void __launch_bounds__(192, 1)
     const int qblk = half ? qb1 : qb0;
     const int t = qblk * kBlock + (r & 63);      // token index of this row
     const uint32_t lane_addr = tbase + ((uint32_t)(quarter * 32) << 16);
-    const float sq = I8 ? prm.sq[bh * prm.nB + min(qblk, prm.nB - 1)] : 1.0f;
+    float sq = 1.0f;
+    if constexpr (I8) sq = prm.sq[bh * prm.nB + min(qblk, prm.nB - 1)];
     float m_run = -INFINITY, l_run = 0.f;
+    // the S tile starts free (INT8: at the magic-number start value)
+    if constexpr (I8) {
+      uint32_t mg[32];
+#pragma unroll
+      for (int i = 0; i < 32; ++i) mg[i] = kMagicBits;
+      tmem_st32(lane_addr + C::S_COL, mg);
+      tmem_st32(lane_addr + C::S_COL + 32, mg);
+      tmem_wait_st();
+    }
+    tc_fence_before();
+    mbar_arrive(&bar_sfree);
     UnionWalk uw;
     uw.init(m0, m1, nW);
     bool ok = true;
@@ -277,51 +291,74 @@ __global__ void __launch_bounds__(192, 1)
     for (int c = 0; c < n; ++c) {
       uw.next(j, fl);
       const int bsel = c & 1;
-      ok = mbar_wait(&bar_sfull[bsel], (c >> 1) & 1, &abort_flag, prm.limit_ns);
+      ok = mbar_wait(&bar_sfull, c & 1, &abort_flag, prm.limit_ns);
       if (!ok) break;
       tc_fence_after();
-      uint32_t sv_raw[64];
+      uint32_t sv[64];
       {
-        uint32_t (&lo)[32] = *reinterpret_cast<uint32_t(*)[32]>(&sv_raw[0]);
-        uint32_t (&hi)[32] = *reinterpret_cast<uint32_t(*)[32]>(&sv_raw[32]);
-        tmem_ld32(lane_addr + C::S_COL + bsel * 64, lo);
-        tmem_ld32(lane_addr + C::S_COL + bsel * 64 + 32, hi);
+        uint32_t (&lo)[32] = *reinterpret_cast<uint32_t(*)[32]>(&sv[0]);
+        uint32_t (&hi)[32] = *reinterpret_cast<uint32_t(*)[32]>(&sv[32]);
+        tmem_ld32(lane_addr + C::S_COL, lo);
+        tmem_ld32(lane_addr + C::S_COL + 32, hi);
         tmem_wait_ld();
       }
+      // hand the S tile back at once (INT8: restarted at the magic value) so the
+      // next S = QK^T runs on the tensor core while this block's softmax runs
+      if constexpr (I8) {
+        uint32_t mg[32];
+#pragma unroll
+        for (int i = 0; i < 32; ++i) mg[i] = kMagicBits;
+        tmem_st32(lane_addr + C::S_COL, mg);
+        tmem_st32(lane_addr + C::S_COL + 32, mg);
+        tmem_wait_st();
+      }
       tc_fence_before();
-      mbar_arrive(&bar_sfree[bsel]);
+      mbar_arrive(&bar_sfree);
       const bool use = ((fl >> half) & 1) != 0;
       const int nvalid = (j == prm.nB - 1) ? (prm.L - j * kBlock) : kBlock;
       float sc = prm.scale_log2;
-      if (I8) sc *= sq * prm.sk[bh * prm.nB + j];
+      if constexpr (I8) sc *= sq * prm.sk[bh * prm.nB + j];
       float m_new = m_run, alpha = 1.f, psum = 0.f;
-      uint32_t pk[I8 ? 16 : 32];
+      constexpr int PW = C::P_COLS;
+      uint32_t pk[PW];
       if (use) {
-        float mx = -INFINITY;
-        if (I8) {
-          int imx = INT32_MIN;
+        // block max (scores read as floats; INT8 ones carry the magic offset)
+        float mx;
+        if (nvalid == kBlock) {
+          float t8[8];
 #pragma unroll
-          for (int u = 0; u < 64; ++u)
-            if (u < nvalid) imx = max(imx, (int)sv_raw[u]);
-          mx = (float)imx * sc;
+          for (int i = 0; i < 8; ++i) t8[i] = __uint_as_float(sv[i]);
+#pragma unroll
+          for (int u = 8; u < 64; ++u) t8[u & 7] = fmaxf(t8[u & 7], __uint_as_float(sv[u]));
+          mx = fmaxf(fmaxf(fmaxf(t8[0], t8[1]), fmaxf(t8[2], t8[3])), fmaxf(fmaxf(t8[4], t8[5]), fmaxf(t8[6], t8[7])));
         } else {
+          mx = -INFINITY;
 #pragma unroll
           for (int u = 0; u < 64; ++u)
-            if (u < nvalid) mx = fmaxf(mx, __uint_as_float(sv_raw[u]));
-          mx *= sc;
+            if (u < nvalid) mx = fmaxf(mx, __uint_as_float(sv[u]));
         }
-        m_new = fmaxf(m_run, mx);
+        const float mblk = (I8 ? (mx - kMagic) : mx) * sc;
+        m_new = fmaxf(m_run, mblk);
         alpha = (m_run == -INFINITY) ? 0.f : ex2f(m_run - m_new);
-        // I8: exponent carries log2(448) so P lands on [0, 448] before the E4M3 cast
-        const float moff = I8 ? (m_new - 8.807354922057604f) : m_new;
+        // exponent argument x = s*sc - m (INT8: P lands on [0, 448] for the E4M3 cast)
+        const float moff = I8 ? (m_new - kLog2_448) : m_new;
+        const uint64_t sc2 = f2pack(sc, sc), nm2 = f2pack(-moff, -moff);
+        const uint64_t mg2 = f2pack(-kMagic, -kMagic);
+        uint64_t acc2 = f2pack(0.f, 0.f);
 #pragma unroll
         for (int u = 0; u < 64; u += 2) {
-          float s0 = I8 ? (float)(int)sv_raw[u] : __uint_as_float(sv_raw[u]);
-          float s1 = I8 ? (float)(int)sv_raw[u + 1] : __uint_as_float(sv_raw[u + 1]);
-          float p0 = u < nvalid ? ex2f(fmaf(s0, sc, -moff)) : 0.f;
-          float p1 = u + 1 < nvalid ? ex2f(fmaf(s1, sc, -moff)) : 0.f;
-          psum += p0 + p1;
-          if (I8) {
+          uint64_t s2 = f2pack(__uint_as_float(sv[u]), __uint_as_float(sv[u + 1]));
+          if constexpr (I8) s2 = add2(s2, mg2);  // exact: the integer score as a float
+          const uint64_t x2 = fma2(s2, sc2, nm2);
+          float x0, x1;
+          f2unpack(x2, x0, x1);
+          float p0 = ex2f(x0), p1 = ex2f(x1);
+          if (nvalid < kBlock) {
+            p0 = u < nvalid ? p0 : 0.f;
+            p1 = u + 1 < nvalid ? p1 : 0.f;
+          }
+          acc2 = add2(acc2, f2pack(p0, p1));
+          if constexpr (I8) {
             const uint32_t e = e4m3x2(p0, p1);
             if ((u & 2) == 0) pk[u >> 2] = e;
             else pk[u >> 2] |= e << 16;
@@ -330,44 +367,46 @@ __global__ void __launch_bounds__(192, 1)
             pk[u >> 1] = *reinterpret_cast<uint32_t*>(&hb);
           }
         }
+        float a0, a1;
+        f2unpack(acc2, a0, a1);
+        psum = a0 + a1;
       } else {
 #pragma unroll
-        for (int i = 0; i < (I8 ? 16 : 32); ++i) pk[i] = 0u;
+        for (int i = 0; i < PW; ++i) pk[i] = 0u;
       }
-      // PV of the previous block must be complete before O or the P buffer is touched
       if (c >= 1) {
+        // PV of the previous block is complete: O may be rescaled and the P
+        // buffer of block c-2 is free again
         ok = mbar_wait(&bar_odone, (c - 1) & 1, &abort_flag, prm.limit_ns);
         if (!ok) break;
         tc_fence_after();
-      }
-      const bool need_rescale = use && c >= 1 && m_run != -INFINITY && m_new > m_run;
-      if (__any_sync(0xffffffffu, need_rescale)) {
-        const float f = need_rescale ? alpha : 1.f;
+        const bool need_rescale = use && m_run != -INFINITY && m_new > m_run;
+        if (__any_sync(0xffffffffu, need_rescale)) {
+          const float f = need_rescale ? alpha : 1.f;
 #pragma unroll
-        for (int cc = 0; cc < D; cc += 32) {
-          uint32_t o[32];
-          tmem_ld32(lane_addr + C::O_COL + cc, o);
-          tmem_wait_ld();
+          for (int cc = 0; cc < D; cc += 32) {
+            uint32_t o[32];
+            tmem_ld32(lane_addr + C::O_COL + cc, o);
+            tmem_wait_ld();
 #pragma unroll
-          for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * f);
-          tmem_st32(lane_addr + C::O_COL + cc, o);
+            for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * f);
+            tmem_st32(lane_addr + C::O_COL + cc, o);
+          }
         }
-        tmem_wait_st();
       }
+      // P of this block into its TMEM buffer: the A operand of PV
+      if constexpr (I8) {
+        tmem_st16(lane_addr + C::P_COL + bsel * C::P_COLS, pk);
+      } else {
+        tmem_st32(lane_addr + C::P_COL + bsel * C::P_COLS, *reinterpret_cast<uint32_t(*)[32]>(pk));
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(&bar_pfull[bsel]);
       if (use) {
         l_run = l_run * alpha + psum;
         m_run = m_new;
       }
-      // write P row (K-major, swizzled) for the PV MMA
-      uint8_t* prow = sm + C::OFF_P + bsel * C::P_BYTES;
-#pragma unroll
-      for (int ch = 0; ch < C::P_ROWB / 16; ++ch) {
-        const uint4 v4 = make_uint4(pk[4 * ch], pk[4 * ch + 1], pk[4 * ch + 2], pk[4 * ch + 3]);
-        *reinterpret_cast<uint4*>(prow + swz_offset(r, ch, C::P_ROWB)) = v4;
-      }
-      fence_proxy_async_smem();
-      tc_fence_before();
-      mbar_arrive(&bar_pfull[bsel]);
     }
     if (!ok) {
       abort_flag = 1;
@@ -393,7 +432,7 @@ __global__ void __launch_bounds__(192, 1)
 #pragma unroll
             for (int i = 0; i < 32; i += 2) {
               float f0 = __uint_as_float(o[i]) * inv_l, f1 = __uint_as_float(o[i + 1]) * inv_l;
-              if (I8) {
+              if constexpr (I8) {
                 f0 *= prm.sv[bh * D + cc + i];
                 f1 *= prm.sv[bh * D + cc + i + 1];
               }

@@ -15,7 +15,7 @@
 namespace {
 
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;  // bound on every device-side wait
-constexpr int64_t kMaxPlannerNB = 2432;                       // score rows of 16 x nB fp32 in shared memory
+constexpr int64_t kMaxPlannerNB = 2176;                       // score rows of 16 x nB fp32 in shared memory
 
 inline bool al16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 inline int64_t n_blocks(int64_t L) { return (L + LX_BLOCK - 1) / LX_BLOCK; }
@@ -103,13 +103,14 @@ template <int D>
 lx_status launch_score(const float* mq, const float* mk, int64_t BH, int64_t nB, int64_t k, lx_plan* plan,
                        cudaStream_t s) {
   const int ldS = (int)((nB + 31) / 32 * 32);
-  const size_t smem = sizeof(float) * ((size_t)lx::kScoreRows * ldS + (size_t)lx::kKeyChunk * D + 8 * 256 +
-                                       2 * 8 * lx::kCandCap + 8 * (ldS / 32));
+  const size_t smem = sizeof(float) * ((size_t)lx::kKeyStages * lx::kKeyChunk * D + (size_t)lx::kScoreRows * ldS +
+                                       lx::kScoreWarps * (256 + 2 * lx::kCandCap + ldS / 32));
+  if (smem > 227 * 1024) return LX_ERR_UNSUPPORTED;
   if (cudaFuncSetAttribute(lx::score_topk_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
       cudaSuccess)
     return LX_ERR_CUDA;
   dim3 grid((unsigned)((nB + lx::kScoreRows - 1) / lx::kScoreRows), (unsigned)BH);
-  lx::score_topk_kernel<D><<<grid, 256, smem, s>>>(mq, mk, (int)nB, (int)k, plan->idx, plan->mask, ldS);
+  lx::score_topk_kernel<D><<<grid, 32 * lx::kScoreWarps, smem, s>>>(mq, mk, (int)nB, (int)k, plan->idx, plan->mask, ldS, kWaitLimitNs);
   return launch_status();
 }
 

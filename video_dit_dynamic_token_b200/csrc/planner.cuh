@@ -87,8 +87,9 @@ __global__ void __launch_bounds__(256) pool_means_kernel(BhldView q, BhldView k,
 }
 
 // ---------------------------------------------------------------------------
-// a2: one CTA per (b*h, 16 query-block rows), 8 warps.
-//  Scoring: every warp computes all 16 rows for its share of the key blocks.
+// a2: one CTA per (b*h, 16 query-block rows), 16 warps.
+//  Scoring: every warp computes all 16 rows for its share of the key blocks
+//  (two keys at a time, so eight independent FMA chains per lane).
 //  Lane = (row group rg in 0..3) x (d-slice ds in 0..7); a lane keeps the 4
 //  rows x D/8 pooled-query values of its slice in registers and reads the
 //  pooled key in 16-byte pieces (slices are interleaved so the 8 slices of one
@@ -109,13 +110,23 @@ __device__ __forceinline__ uint32_t lanemask_lt() {
   return m;
 }
 
+// Pooled keys stream through a ring of shared-memory stages filled by bulk
+// copies (one thread issues, every warp reads), so the L2 latency of one chunk
+// hides behind the arithmetic on the previous ones.
+constexpr int kKeyStages = 3;
+constexpr int kScoreWarps = 16;  // 512 threads share one CTA's score rows
+
 template <int D>
 __device__ __forceinline__ void score_rows(const float* __restrict__ Mq, const float* __restrict__ Mk, int nB,
-                                           int row0, int nrows, float* sS, int ldS, float* sK) {
+                                           int row0, int nrows, float* sS, int ldS, float* sK, uint64_t* kfull,
+                                           uint64_t* kempty, const volatile int* abort_flag,
+                                           unsigned long long limit_ns) {
   constexpr int DS = D / 8;   // values per lane slice
   constexpr int NQ = DS / 4;  // float4 pieces per slice
+  constexpr int CHUNK_FLOATS = kKeyChunk * D;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int rg = lane >> 3, ds = lane & 7;
+  const int nchunks = (nB + kKeyChunk - 1) / kKeyChunk;
   // Slice ds covers d = 32*qq + 4*ds + e  (qq < NQ, e < 4).
   float qv[4][DS];
 #pragma unroll
@@ -131,45 +142,76 @@ __device__ __forceinline__ void score_rows(const float* __restrict__ Mq, const f
       qv[r][4 * qq + 3] = v.w;
     }
   }
-  for (int j0 = 0; j0 < nB; j0 += kKeyChunk) {
+  auto issue = [&](int ch) {
+    const int st = ch % kKeyStages;
+    const int nk = min(kKeyChunk, nB - ch * kKeyChunk);
+    mbar_arrive_expect_tx(&kfull[st], (uint32_t)(nk * D * 4));
+    bulk_load(sK + st * CHUNK_FLOATS, Mk + (long long)ch * kKeyChunk * D, (uint32_t)(nk * D * 4), &kfull[st]);
+  };
+  if (threadIdx.x == 0)
+    for (int ch = 0; ch < min(kKeyStages, nchunks); ++ch) issue(ch);
+  bool ok = true;
+  for (int ch = 0; ch < nchunks; ++ch) {
+    const int st = ch % kKeyStages;
+    const int j0 = ch * kKeyChunk;
     const int nk = min(kKeyChunk, nB - j0);
-    __syncthreads();  // previous chunk fully consumed
-    for (int e = threadIdx.x; e < nk * (D / 4); e += blockDim.x) {
-      const int jj = e / (D / 4), d4 = e % (D / 4);
-      reinterpret_cast<float4*>(sK)[e] = *reinterpret_cast<const float4*>(Mk + (long long)(j0 + jj) * D + 4 * d4);
-      (void)jj;
+    if (!mbar_wait(&kfull[st], (ch / kKeyStages) & 1, abort_flag, limit_ns)) {
+      ok = false;
+      break;
     }
-    __syncthreads();
-    // warp w handles keys jj = w, w+8, w+16, w+24 of the chunk
-    for (int jj = warp; jj < nk; jj += 8) {
-      const float* kr = sK + jj * D;
-      float acc[4] = {0.f, 0.f, 0.f, 0.f};
+    const float* sKc = sK + st * CHUNK_FLOATS;
+    // warp w handles keys jj = w and w + 16 of the chunk, together
+    {
+      const int ja = warp, jb = warp + kScoreWarps;
+      const bool va = ja < nk, vb = jb < nk;
+      const float* ka = sKc + (va ? ja : 0) * D;
+      const float* kb = sKc + (vb ? jb : 0) * D;
+      float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
 #pragma unroll
       for (int qq = 0; qq < NQ; ++qq) {
-        const float4 kv = *reinterpret_cast<const float4*>(kr + 32 * qq + 4 * ds);
+        const float4 xa = *reinterpret_cast<const float4*>(ka + 32 * qq + 4 * ds);
+        const float4 xb = *reinterpret_cast<const float4*>(kb + 32 * qq + 4 * ds);
 #pragma unroll
         for (int r = 0; r < 4; ++r) {
-          acc[r] = fmaf(qv[r][4 * qq], kv.x, acc[r]);
-          acc[r] = fmaf(qv[r][4 * qq + 1], kv.y, acc[r]);
-          acc[r] = fmaf(qv[r][4 * qq + 2], kv.z, acc[r]);
-          acc[r] = fmaf(qv[r][4 * qq + 3], kv.w, acc[r]);
+          acc[0][r] = fmaf(qv[r][4 * qq], xa.x, acc[0][r]);
+          acc[1][r] = fmaf(qv[r][4 * qq], xb.x, acc[1][r]);
+          acc[0][r] = fmaf(qv[r][4 * qq + 1], xa.y, acc[0][r]);
+          acc[1][r] = fmaf(qv[r][4 * qq + 1], xb.y, acc[1][r]);
+          acc[0][r] = fmaf(qv[r][4 * qq + 2], xa.z, acc[0][r]);
+          acc[1][r] = fmaf(qv[r][4 * qq + 2], xb.z, acc[1][r]);
+          acc[0][r] = fmaf(qv[r][4 * qq + 3], xa.w, acc[0][r]);
+          acc[1][r] = fmaf(qv[r][4 * qq + 3], xb.w, acc[1][r]);
         }
       }
       // fold the 8 slices: after three stages lane ds holds row 2*(ds>>2&1)+(ds>>1&1)
-      const bool hi4 = (ds & 4) != 0;
-      float s0 = hi4 ? acc[0] : acc[2], s1 = hi4 ? acc[1] : acc[3];
-      float k0 = hi4 ? acc[2] : acc[0], k1 = hi4 ? acc[3] : acc[1];
-      k0 += __shfl_xor_sync(0xffffffffu, s0, 4);
-      k1 += __shfl_xor_sync(0xffffffffu, s1, 4);
-      const bool hi2 = (ds & 2) != 0;
-      float s2 = hi2 ? k0 : k1;
-      float k2 = hi2 ? k1 : k0;
-      k2 += __shfl_xor_sync(0xffffffffu, s2, 2);
-      k2 += __shfl_xor_sync(0xffffffffu, k2, 1);
+      const bool hi4 = (ds & 4) != 0, hi2 = (ds & 2) != 0;
       const int r = 2 * (hi4 ? 1 : 0) + (hi2 ? 1 : 0);
-      if ((ds & 1) == 0) sS[(rg * 4 + r) * ldS + j0 + jj] = k2;
+#pragma unroll
+      for (int kx = 0; kx < 2; ++kx) {
+        float s0 = hi4 ? acc[kx][0] : acc[kx][2], s1 = hi4 ? acc[kx][1] : acc[kx][3];
+        float k0 = hi4 ? acc[kx][2] : acc[kx][0], k1 = hi4 ? acc[kx][3] : acc[kx][1];
+        k0 += __shfl_xor_sync(0xffffffffu, s0, 4);
+        k1 += __shfl_xor_sync(0xffffffffu, s1, 4);
+        float s2 = hi2 ? k0 : k1;
+        float k2 = hi2 ? k1 : k0;
+        k2 += __shfl_xor_sync(0xffffffffu, s2, 2);
+        k2 += __shfl_xor_sync(0xffffffffu, k2, 1);
+        const int jj = kx ? jb : ja;
+        if ((ds & 1) == 0 && (kx ? vb : va)) sS[(rg * 4 + r) * ldS + j0 + jj] = k2;
+      }
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&kempty[st]);
+    // refill this stage with chunk ch + kKeyStages once all warps are done with it
+    if (threadIdx.x == 0 && ch + kKeyStages < nchunks) {
+      if (!mbar_wait(&kempty[st], (ch / kKeyStages) & 1, abort_flag, limit_ns)) {
+        ok = false;
+        break;
+      }
+      issue(ch + kKeyStages);
     }
   }
+  if (!ok) report_error(-6);
   __syncthreads();
 }
 
@@ -312,23 +354,36 @@ __device__ int select_row(const float* __restrict__ s, int nB, int k, int* hist,
 }
 
 template <int D>
-__global__ void __launch_bounds__(256, 1) score_topk_kernel(const float* __restrict__ Mq, const float* __restrict__ Mk,
+__global__ void __launch_bounds__(512, 1) score_topk_kernel(const float* __restrict__ Mq, const float* __restrict__ Mk,
                                                            int nB, int k, int32_t* __restrict__ idx,
-                                                           uint32_t* __restrict__ mask, int ldS) {
+                                                           uint32_t* __restrict__ mask, int ldS,
+                                                           unsigned long long limit_ns) {
   extern __shared__ __align__(16) float smem_f[];
-  float* sS = smem_f;                                  // [16][ldS]
-  float* sK = sS + kScoreRows * ldS;                   // [32][D]
-  int* hist = reinterpret_cast<int*>(sK + kKeyChunk * D);          // 8 x 256
-  float* cand_s = reinterpret_cast<float*>(hist + 8 * 256);       // 8 x 64
-  int* cand_j = reinterpret_cast<int*>(cand_s + 8 * kCandCap);    // 8 x 64
-  uint32_t* selbits = reinterpret_cast<uint32_t*>(cand_j + 8 * kCandCap);  // 8 x ldS/32
+  float* sK = smem_f;                                              // kKeyStages x [32][D]
+  float* sS = sK + kKeyStages * kKeyChunk * D;                     // [16][ldS]
+  int* hist = reinterpret_cast<int*>(sS + kScoreRows * ldS);                 // warps x 256
+  float* cand_s = reinterpret_cast<float*>(hist + kScoreWarps * 256);       // warps x 64
+  int* cand_j = reinterpret_cast<int*>(cand_s + kScoreWarps * kCandCap);    // warps x 64
+  uint32_t* selbits = reinterpret_cast<uint32_t*>(cand_j + kScoreWarps * kCandCap);  // warps x ldS/32
+  __shared__ uint64_t kfull[kKeyStages], kempty[kKeyStages];
+  __shared__ int never_abort;
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kKeyStages; ++i) {
+      mbar_init(&kfull[i], 1);
+      mbar_init(&kempty[i], kScoreWarps);
+    }
+    never_abort = 0;
+    fence_barrier_init();
+  }
+  __syncthreads();
   const long long bh = blockIdx.y;
   const int row0 = blockIdx.x * kScoreRows;
   const int nrows = min(kScoreRows, nB - row0);
-  score_rows<D>(Mq + bh * nB * D, Mk + bh * nB * D, nB, row0, nrows, sS, ldS, sK);
+  score_rows<D>(Mq + bh * nB * D, Mk + bh * nB * D, nB, row0, nrows, sS, ldS, sK, kfull, kempty, &never_abort,
+                limit_ns);
   const int warp = threadIdx.x >> 5;
   const int nW = (nB + 31) >> 5;
-  for (int r = warp; r < nrows; r += 8) {
+  for (int r = warp; r < nrows; r += kScoreWarps) {
     const long long row = bh * nB + row0 + r;
     const int got = select_row(sS + r * ldS, nB, k, hist + warp * 256, cand_s + warp * kCandCap,
                                cand_j + warp * kCandCap, selbits + warp * (ldS / 32), idx + row * k,
