@@ -43,7 +43,7 @@ struct AttnCfg {
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_K = OFF_Q + Q_BYTES;
   static constexpr int OFF_V = OFF_K + NSTAGE * KV_BYTES;
-  static constexpr int OFF_MASK = OFF_V + NSTAGE * KV_BYTES;  // two bitmask rows follow
+  static constexpr int OFF_MASK = OFF_V + NSTAGE * KV_BYTES;  // two bitmask rows, then (INT8) the K block scales
   static constexpr int P_COLS = 64 * ESZ / 4;             // P of one 64-key block: 16 (E4M3) or 32 (bf16) cols
   static constexpr int S_COL = 0;                         // TMEM: S tile, cols [0, 64)
   static constexpr int P_COL = 64;                        // TMEM: two P buffers, P_COLS each
@@ -129,6 +129,7 @@ __global__ void __launch_bounds__(192, I8 ? 2 : 1)
   const int nW = (prm.nB + 31) >> 5;
   uint32_t* m0 = reinterpret_cast<uint32_t*>(sm + C::OFF_MASK);
   uint32_t* m1 = m0 + nW;
+  float* sk_s = reinterpret_cast<float*>(m1 + nW);  // INT8: this head's K block scales
 
   // ---- prologue: barriers, kept-list bitmasks (validated), TMEM
   if (threadIdx.x == 0) {
@@ -147,6 +148,8 @@ __global__ void __launch_bounds__(192, I8 ? 2 : 1)
     fence_barrier_init();
   }
   for (int w = threadIdx.x; w < 2 * nW; w += blockDim.x) m0[w] = 0u;
+  if constexpr (I8)
+    for (int jj = threadIdx.x; jj < prm.nB; jj += blockDim.x) sk_s[jj] = prm.sk[bh * prm.nB + jj];
   __syncthreads();
   {
     const int32_t* r0 = prm.idx + (bh * prm.nB + qb0) * (long long)prm.k;
@@ -317,7 +320,7 @@ __global__ void __launch_bounds__(192, I8 ? 2 : 1)
       const bool use = ((fl >> half) & 1) != 0;
       const int nvalid = (j == prm.nB - 1) ? (prm.L - j * kBlock) : kBlock;
       float sc = prm.scale_log2;
-      if constexpr (I8) sc *= sq * prm.sk[bh * prm.nB + j];
+      if constexpr (I8) sc *= sq * sk_s[j];
       float m_new = m_run, alpha = 1.f, psum = 0.f;
       constexpr int PW = C::P_COLS;
       uint32_t pk[PW];
@@ -344,7 +347,8 @@ __global__ void __launch_bounds__(192, I8 ? 2 : 1)
         const float moff = I8 ? (m_new - kLog2_448) : m_new;
         const uint64_t sc2 = f2pack(sc, sc), nm2 = f2pack(-moff, -moff);
         const uint64_t mg2 = f2pack(-kMagic, -kMagic);
-        uint64_t acc2 = f2pack(0.f, 0.f);
+        uint64_t acc2[4] = {f2pack(0.f, 0.f), f2pack(0.f, 0.f), f2pack(0.f, 0.f), f2pack(0.f, 0.f)};
+        const bool partial = nvalid < kBlock;
 #pragma unroll
         for (int u = 0; u < 64; u += 2) {
           uint64_t s2 = f2pack(__uint_as_float(sv[u]), __uint_as_float(sv[u + 1]));
@@ -352,12 +356,18 @@ __global__ void __launch_bounds__(192, I8 ? 2 : 1)
           const uint64_t x2 = fma2(s2, sc2, nm2);
           float x0, x1;
           f2unpack(x2, x0, x1);
-          float p0 = ex2f(x0), p1 = ex2f(x1);
-          if (nvalid < kBlock) {
-            p0 = u < nvalid ? p0 : 0.f;
-            p1 = u + 1 < nvalid ? p1 : 0.f;
-          }
-          acc2 = add2(acc2, f2pack(p0, p1));
+          sv[u] = __float_as_uint(ex2f(x0));
+          sv[u + 1] = __float_as_uint(ex2f(x1));
+        }
+        if (partial) {
+#pragma unroll
+          for (int u = 0; u < 64; ++u)
+            if (u >= nvalid) sv[u] = 0u;
+        }
+#pragma unroll
+        for (int u = 0; u < 64; u += 2) {
+          const float p0 = __uint_as_float(sv[u]), p1 = __uint_as_float(sv[u + 1]);
+          acc2[(u >> 1) & 3] = add2(acc2[(u >> 1) & 3], f2pack(p0, p1));
           if constexpr (I8) {
             const uint32_t e = e4m3x2(p0, p1);
             if ((u & 2) == 0) pk[u >> 2] = e;
@@ -367,9 +377,12 @@ __global__ void __launch_bounds__(192, I8 ? 2 : 1)
             pk[u >> 1] = *reinterpret_cast<uint32_t*>(&hb);
           }
         }
-        float a0, a1;
-        f2unpack(acc2, a0, a1);
-        psum = a0 + a1;
+        float a0, a1, a2, a3, b0, b1, b2, b3;
+        f2unpack(acc2[0], a0, b0);
+        f2unpack(acc2[1], a1, b1);
+        f2unpack(acc2[2], a2, b2);
+        f2unpack(acc2[3], a3, b3);
+        psum = ((a0 + b0) + (a1 + b1)) + ((a2 + b2) + (a3 + b3));
       } else {
 #pragma unroll
         for (int i = 0; i < PW; ++i) pk[i] = 0u;
