@@ -116,6 +116,35 @@ lx_status lx_quantize_qk(const lx_bhld* Q, const lx_bhld* K, int8_t* qc, float* 
  * amax_ws: caller scratch of B*H*D uint32 (zeroed by the call). */
 lx_status lx_quantize_v(const lx_bhld* V, uint8_t* vc, float* vs, uint32_t* amax_ws, cudaStream_t stream);
 
+/* Largest B*H*D that lx_quantize_v_noalloc accepts (its built-in scratch holds
+ * this many uint32 words, 256 KiB per device). */
+#define LX_NOALLOC_AMAX_MAX 65536
+
+/* lx_quantize_v without a caller-supplied scratch buffer.  The paper has no
+ * counterpart to this call: it exists for callers that cannot hand over device
+ * scratch, e.g. plain C hosts without a device allocator of their own, where a
+ * cudaMalloc/cudaFree pair per call would synchronise the device, or callers
+ * whose device memory is fully budgeted up front.  It computes exactly what
+ * lx_quantize_v computes (same codes and scales, bit for bit) and allocates
+ * nothing.
+ *
+ * Scratch: a per-device array of LX_NOALLOC_AMAX_MAX uint32 words built into
+ * this library.  The call zeroes the first B*H*D words on `stream` before use,
+ * so nothing has to be cleared beforehand.  Because the array is shared, calls
+ * that may overlap on the same device (two streams, two host threads without
+ * ordering) race on it and may produce wrong scales; serialise them, or use
+ * lx_quantize_v with a buffer per stream.
+ *
+ * First-call setup: the first call on each device looks up the array's device
+ * address (cudaGetSymbolAddress, with that device current, guarded by a host
+ * mutex) and caches it; later calls only read the cache.  That lookup may load
+ * the library's device code, so make the first call on a device before any
+ * stream capture begins.
+ *
+ * Errors: LX_ERR_WORKSPACE when B*H*D > LX_NOALLOC_AMAX_MAX (nothing is
+ * launched); LX_ERR_CUDA when the lookup fails; otherwise as lx_quantize_v. */
+lx_status lx_quantize_v_noalloc(const lx_bhld* V, uint8_t* vc, float* vs, cudaStream_t stream);
+
 /* Step a4 -- attention over the kept blocks in BF16 (tcgen05 kind::f16).
  * O[t] = sum_u softmax_u(q_t.k_u/sqrt(D)) v_u over the valid keys u of the
  * kept blocks of t's query block ("600倍加速…", §动态稀疏量化注意力). */

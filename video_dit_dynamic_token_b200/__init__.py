@@ -152,6 +152,18 @@ def lx_quantize_v(V, out=None, amax_ws=None, stream=None):
     return out
 
 
+def lx_quantize_v_noalloc(V, out=None, stream=None):
+    lib = _abi.load()
+    B, H, L, D = V.shape
+    if out is None:
+        out = (torch.empty((B, H, L, D), dtype=torch.uint8, device=V.device),
+               torch.empty((B, H, D), dtype=torch.float32, device=V.device))
+    v = bhld(V)
+    _check(lib.lx_quantize_v_noalloc(ctypes.byref(v), _ptr(out[0]), _ptr(out[1]), _stream(stream)),
+           "lx_quantize_v_noalloc")
+    return out
+
+
 def lx_attn_bf16(Q, K, V, plan: Plan, out=None, stream=None):
     lib = _abi.load()
     if out is None:

@@ -18,6 +18,7 @@ LX_ERR_PLAN = -7
 LX_MODE_BF16 = 0
 LX_MODE_INT8FP8 = 1
 LX_BLOCK = 64
+LX_NOALLOC_AMAX_MAX = 65536
 
 # every entry point the header declares, with its ctypes signature
 _c_i64, _c_sz, _vp, _dbl, _u64 = ctypes.c_int64, ctypes.c_size_t, ctypes.c_void_p, ctypes.c_double, ctypes.c_uint64
@@ -41,6 +42,7 @@ SIGNATURES = {
     "lx_sparse_attn_plan": [_P(LxBhld), _P(LxBhld), _dbl, _P(LxPlan), _vp, _c_sz, _vp],
     "lx_quantize_qk": [_P(LxBhld), _P(LxBhld), _vp, _vp, _vp, _vp, _vp],
     "lx_quantize_v": [_P(LxBhld), _vp, _vp, _vp, _vp],
+    "lx_quantize_v_noalloc": [_P(LxBhld), _vp, _vp, _vp],
     "lx_attn_bf16": [_P(LxBhld), _P(LxBhld), _P(LxBhld), _P(LxPlan), _P(LxBhld), _vp],
     "lx_attn_int8fp8": [_vp, _vp, _vp, _vp, _vp, _vp, _P(LxPlan), _P(LxBhld), _vp],
     "lx_fwd_workspace_size": [_P(LxBhld), ctypes.c_int, _P(_c_sz)],

@@ -5,6 +5,7 @@
 #include <cmath>
 #include <cstdint>
 #include <cstring>
+#include <mutex>
 
 #include "lx_sparse_attn.h"
 #include "ptx.cuh"
@@ -301,6 +302,41 @@ lx_status lx_quantize_v(const lx_bhld* V, uint8_t* vc, float* vs, uint32_t* amax
   if (!al16(vc) || !al16(vs) || !al16(amax_ws)) return LX_ERR_ALIGN;
   return V->D == 128 ? launch_quant_v<128>(V, vc, vs, amax_ws, stream)
                      : launch_quant_v<64>(V, vc, vs, amax_ws, stream);
+}
+
+// Built-in V absmax scratch of lx_quantize_v_noalloc (one copy per device).
+static __device__ __align__(256) uint32_t g_noalloc_amax[LX_NOALLOC_AMAX_MAX];
+
+namespace {
+constexpr int kMaxDevices = 64;
+std::mutex g_noalloc_mu;
+uint32_t* g_noalloc_ptr[kMaxDevices] = {};
+
+// Device address of g_noalloc_amax on the current device, looked up once.
+lx_status noalloc_scratch(uint32_t** out) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) return LX_ERR_CUDA;
+  if (dev >= kMaxDevices) return LX_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (!g_noalloc_ptr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_amax) != cudaSuccess || !p) return LX_ERR_CUDA;
+    g_noalloc_ptr[dev] = static_cast<uint32_t*>(p);
+  }
+  *out = g_noalloc_ptr[dev];
+  return LX_OK;
+}
+}  // namespace
+
+lx_status lx_quantize_v_noalloc(const lx_bhld* V, uint8_t* vc, float* vs, cudaStream_t stream) {
+  lx_status st = check_bhld(V);
+  if (st != LX_OK) return st;
+  if (!vc || !vs) return LX_ERR_INVALID;
+  if (!al16(vc) || !al16(vs)) return LX_ERR_ALIGN;
+  if (V->B * V->H * V->D > (int64_t)LX_NOALLOC_AMAX_MAX) return LX_ERR_WORKSPACE;
+  uint32_t* amax = nullptr;
+  if ((st = noalloc_scratch(&amax)) != LX_OK) return st;
+  return V->D == 128 ? launch_quant_v<128>(V, vc, vs, amax, stream) : launch_quant_v<64>(V, vc, vs, amax, stream);
 }
 
 lx_status lx_attn_bf16(const lx_bhld* Q, const lx_bhld* K, const lx_bhld* V, const lx_plan* plan, const lx_bhld* O,
