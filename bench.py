@@ -29,6 +29,29 @@ MODE = "int8fp8"
 METRIC = "block-sparse attn effective TFLOPS (720p grid, 40x128, keep 10%)"
 
 
+# DRAM bytes (read + write) of one full-size attention launch of the current
+# kernel build: the ncu capture in profiles/attn_int8fp8_720p_8heads_ncu.md
+# (8 of the 40 heads; traffic grows with the head count, so x5).  Set to None
+# whenever the attention kernel changes until it is captured again.
+ATTN_DRAM_BYTES_PER_LAUNCH = 5 * (237.007360e6 + 127.056384e6)
+
+
+def reduce_max(x: float, device) -> float:
+    """Max of a per-rank float over all ranks (the job's time is its slowest rank's)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(x)
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_tflops(world: int, flops_per_rank: float, ms_per_step: float) -> float:
+    """Whole-job throughput: every rank processes its own batch of `flops_per_rank`."""
+    return world * flops_per_rank / (ms_per_step * 1e-3) / 1e12
+
+
 def _peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -173,12 +196,9 @@ def run_ours(args, rank, world, local_rank):
     if lx.lx_last_device_status() != 0:
         raise RuntimeError("device status error in timed region")
 
-    if world > 1:
-        t = torch.tensor([total_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = reduce_max(total_ms, dev)
     ms_step = total_ms / args.steps
-    value = world * flops / (ms_step * 1e-3) / 1e12
+    value = job_tflops(world, flops, ms_step)
 
     # ---- end to end through the public API with host buffers
     e2e = None
@@ -206,12 +226,8 @@ def run_ours(args, rank, world, local_rank):
             e2e_step()
         b.record(stream)
         torch.cuda.synchronize()
-        e_ms = a.elapsed_time(b) / args.e2e_steps
-        if world > 1:
-            t = torch.tensor([e_ms], device=dev)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            e_ms = float(t.item())
-        e2e = {"value": world * flops / (e_ms * 1e-3) / 1e12, "unit": "TFLOP/s", "ms_per_step": e_ms,
+        e_ms = reduce_max(a.elapsed_time(b) / args.e2e_steps, dev)
+        e2e = {"value": job_tflops(world, flops, e_ms), "unit": "TFLOP/s", "ms_per_step": e_ms,
                "h2d_bytes_per_step": 3 * Q.numel() * 2, "d2h_bytes_per_step": O.numel() * 2}
 
     if rank != 0:
@@ -222,6 +238,8 @@ def run_ours(args, rank, world, local_rank):
     peak = 2.0 * peaks["bf16_sustained"]
     plan_bytes = 2 * B * H * L * d * 2 + B * H * nB * k * 4 + B * H * nB * ((nB + 31) // 32) * 4
     plan_ms = per["pool"] + per["score_topk"]
+    # Q/K/V codes read once, O written once (bf16), kept ids
+    attn_bytes = 3 * B * H * L * d + B * H * L * d * 2 + B * H * nB * k * 4
     out = {
         "metric": METRIC, "value": round(value, 2), "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(ms_step, 4), "higher_is_better": True, "scaling": "weak",
@@ -237,7 +255,10 @@ def run_ours(args, rank, world, local_rank):
                      "peak": round(peak, 1), "unit": "TFLOP/s", "frac": round(achieved / peak, 3),
                      "peak_note": f"2 x {peaks['source']} sustained bf16 ({peaks['bf16_sustained']}) = dense "
                                   "int8/fp8 by the nominal 2:1 ratio",
-                     "traffic": None},
+                     "traffic": (None if ATTN_DRAM_BYTES_PER_LAUNCH is None or args.heads
+                                 else int(ATTN_DRAM_BYTES_PER_LAUNCH)),
+                     "traffic_note": "ncu dram__bytes_read+write per launch (8-head capture x5)",
+                     "algorithmic_bytes": int(attn_bytes)},
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clocks,
         "e2e": e2e,
