@@ -5,17 +5,22 @@
 // inside; §高效推理算子: Q/K INT8 and V FP8.  "Run Wan2.2-A14B on One RTX 5090:
 // 720p Video in 3.8s", §3 Dynamic sparse attention: the same in English.
 //
-// Tile: one CTA owns two adjacent 64-row query blocks (2p, 2p+1) = 128 rows,
-// the full-rate M of a single-CTA tcgen05 MMA, and walks the ascending UNION of
-// their two kept lists one 64-key block at a time.  A row whose own list does
-// not hold the current block gets P = 0 for it and leaves its running max and
-// sum untouched, so every row sees exactly its kept blocks in ascending order.
+// Tile: one CTA owns two adjacent 64-row query blocks (2p, 2p+1), run as two
+// independent M=64 streams A and B in lockstep.  Step c computes query block
+// 2p against its c-th kept key block and query block 2p+1 against ITS c-th
+// kept key block, so every row works on one of its own kept blocks at every
+// step and a CTA takes exactly k steps (no union of the two lists, no idle
+// rows).  The two M=64 accumulators of a step share TMEM columns: stream A in
+// lanes 0-15 and stream B in lanes 16-31 of each 32-lane subpartition (the
+// half-subpartition layout of an M=64 tcgen05 accumulator), so one warp's
+// 32x32b TMEM load returns 16 rows of A and 16 rows of B.
 //
-// Roles (6 warps): warp 0 = TMA producer (Q once, then K/V of each union block
-// into a ring of stages); warp 1 = TMEM allocator + MMA issuer
-// (S = Q K^T into one of two TMEM S buffers, then O += P V into the TMEM O
-// accumulator); warps 2..5 = softmax / correction / epilogue, one thread per
-// query row (a warp reads the TMEM lane quarter warp%4).
+// Roles (6 warps): warp 0 = TMA producer (Q once; K blocks of both streams
+// into a 3-stage ring, V blocks into a 2-stage ring); warp 1 = TMEM allocator
+// + MMA issuer (S_A, S_B = Q K^T into the S columns, then O_A, O_B += P V into
+// the O columns, P and V read from shared memory); warps 2..5 = softmax /
+// correction / epilogue, one thread per (stream, row): thread t of warp w
+// reads TMEM lane 32*(w%4) + t, i.e. row 16*(w%4) + t%16 of stream t/16.
 //
 // INT8/FP8 mode follows the P-quantisation protocol: per 64-key block c the
 // row max becomes m_c = max(m_{c-1}, max S_c); P~ = E4M3(448 exp(S_c - m_c));
@@ -36,23 +41,27 @@ struct AttnCfg {
   static constexpr int ROWB = D * ESZ;                    // bytes per token row
   static constexpr int ATOM = ROWB >= 128 ? 128 : ROWB;   // swizzle atom width (128 or 64 bytes)
   static constexpr int NATOM = ROWB / ATOM;               // atom columns per row
-  static constexpr int Q_BYTES = 128 * ROWB;
+  static constexpr int Q_BYTES = 128 * ROWB;              // rows 0-63: stream A, rows 64-127: stream B
   static constexpr int KV_BYTES = 64 * ROWB;              // one K (or V) block
-  static constexpr int NSTAGE = I8 ? 5 : 3;   // INT8: two CTAs fit one SM
+  static constexpr int KSTAGE = 3;                        // K ring (A and B blocks per stage)
+  static constexpr int VSTAGE = 2;                        // V ring (A and B blocks per stage)
+  static constexpr int P_ROWB = 64 * ESZ;                 // P row: 64 keys
+  static constexpr int P_BYTES = 64 * P_ROWB;             // P of one stream, K-major, swizzled
   static constexpr uint32_t SW_QKV = ATOM == 128 ? SW_128B : SW_64B;
+  static constexpr uint32_t SW_P = P_ROWB == 128 ? SW_128B : SW_64B;
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_K = OFF_Q + Q_BYTES;
-  static constexpr int OFF_V = OFF_K + NSTAGE * KV_BYTES;
-  static constexpr int OFF_MASK = OFF_V + NSTAGE * KV_BYTES;  // two bitmask rows, then (INT8) the K block scales
-  static constexpr int P_COLS = 64 * ESZ / 4;             // P of one 64-key block: 16 (E4M3) or 32 (bf16) cols
-  static constexpr int S_COL = 0;                         // TMEM: S tile, cols [0, 64)
-  static constexpr int P_COL = 64;                        // TMEM: two P buffers, P_COLS each
+  static constexpr int OFF_V = OFF_K + KSTAGE * 2 * KV_BYTES;
+  static constexpr int OFF_P = OFF_V + VSTAGE * 2 * KV_BYTES;
+  static constexpr int OFF_IDX = OFF_P + 2 * P_BYTES;     // the two kept lists (2 x k int32) follow
+  static constexpr int S_COL = 0;                         // TMEM: S, cols [0, 64)
   static constexpr int O_COL = 128;                       // TMEM: O accumulator, D cols
+  static constexpr uint32_t LANE_B = 16u << 16;           // TMEM address offset of stream B (lane 16)
   static constexpr uint32_t TMEM_COLS = 256;
   static constexpr uint32_t IDESC_S =
-      instr_desc(I8 ? IDESC_DS32 : IDESC_DF32, I8 ? IDESC_S8 : IDESC_BF16, I8 ? IDESC_S8 : IDESC_BF16, 0, 0, 128, 64);
+      instr_desc(I8 ? IDESC_DS32 : IDESC_DF32, I8 ? IDESC_S8 : IDESC_BF16, I8 ? IDESC_S8 : IDESC_BF16, 0, 0, 64, 64);
   static constexpr uint32_t IDESC_PV =
-      instr_desc(IDESC_DF32, I8 ? IDESC_E4M3 : IDESC_BF16, I8 ? IDESC_E4M3 : IDESC_BF16, 0, 1, 128, D);
+      instr_desc(IDESC_DF32, I8 ? IDESC_E4M3 : IDESC_BF16, I8 ? IDESC_E4M3 : IDESC_BF16, 0, 1, 64, D);
   static constexpr int KEYS_PER_MMA = 32 / ESZ;           // 32 bytes of K per instruction
 };
 
@@ -66,31 +75,6 @@ struct AttnParams {
   const float* sv;        // [B*H, D] V channel scales
   float scale_log2;       // log2(e)/sqrt(d)
   unsigned long long limit_ns;  // bound on every wait
-};
-
-struct UnionWalk {
-  const uint32_t* m0;
-  const uint32_t* m1;
-  int nW, w;
-  uint32_t rem;
-  __device__ __forceinline__ void init(const uint32_t* a, const uint32_t* b, int n) {
-    m0 = a;
-    m1 = b;
-    nW = n;
-    w = 0;
-    rem = n > 0 ? (a[0] | b[0]) : 0u;
-  }
-  __device__ __forceinline__ bool next(int& j, int& flags) {
-    while (rem == 0u) {
-      if (++w >= nW) return false;
-      rem = m0[w] | m1[w];
-    }
-    const int bit = __ffs(rem) - 1;
-    rem &= rem - 1u;
-    j = w * 32 + bit;
-    flags = (int)((m0[w] >> bit) & 1u) | ((int)((m1[w] >> bit) & 1u) << 1);
-    return true;
-  }
 };
 
 __device__ __forceinline__ float ex2f(float x) {
@@ -113,11 +97,10 @@ __global__ void __launch_bounds__(192, I8 ? 2 : 1)
   using C = AttnCfg<D, I8>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  __shared__ uint64_t bar_q, bar_full[C::NSTAGE], bar_empty[C::NSTAGE], bar_sfull, bar_sfree, bar_pfull[2], bar_odone,
-      bar_drain;
+  __shared__ uint64_t bar_q, bar_kfull[C::KSTAGE], bar_kempty[C::KSTAGE], bar_vfull[C::VSTAGE],
+      bar_vempty[C::VSTAGE], bar_sfull, bar_sfree, bar_pfull, bar_odone, bar_drain;
   __shared__ uint32_t tmem_slot;
   __shared__ volatile int abort_flag;
-  __shared__ int n_union;
   __shared__ int never_abort;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -126,44 +109,42 @@ __global__ void __launch_bounds__(192, I8 ? 2 : 1)
   const int b_idx = (int)(bh / prm.H), h_idx = (int)(bh % prm.H);
   const int qb0 = 2 * pair, qb1 = 2 * pair + 1;
   const bool has1 = qb1 < prm.nB;
-  const int nW = (prm.nB + 31) >> 5;
-  uint32_t* m0 = reinterpret_cast<uint32_t*>(sm + C::OFF_MASK);
-  uint32_t* m1 = m0 + nW;
-  float* sk_s = reinterpret_cast<float*>(m1 + nW);  // INT8: this head's K block scales
+  const int n = prm.k;  // steps: every stream walks exactly k kept blocks
+  int32_t* idx0 = reinterpret_cast<int32_t*>(sm + C::OFF_IDX);
+  int32_t* idx1 = idx0 + n;
 
-  // ---- prologue: barriers, kept-list bitmasks (validated), TMEM
+  // ---- prologue: barriers, the two kept lists (validated), TMEM
   if (threadIdx.x == 0) {
     mbar_init(&bar_q, 1);
-    for (int s = 0; s < C::NSTAGE; ++s) {
-      mbar_init(&bar_full[s], 1);
-      mbar_init(&bar_empty[s], 1);
+    for (int s = 0; s < C::KSTAGE; ++s) {
+      mbar_init(&bar_kfull[s], 1);
+      mbar_init(&bar_kempty[s], 1);
+    }
+    for (int s = 0; s < C::VSTAGE; ++s) {
+      mbar_init(&bar_vfull[s], 1);
+      mbar_init(&bar_vempty[s], 1);
     }
     mbar_init(&bar_sfull, 1);
     mbar_init(&bar_sfree, 128);
-    for (int i = 0; i < 2; ++i) mbar_init(&bar_pfull[i], 128);
+    mbar_init(&bar_pfull, 128);
     mbar_init(&bar_odone, 1);
     mbar_init(&bar_drain, 1);
     abort_flag = 0;
     never_abort = 0;
     fence_barrier_init();
   }
-  for (int w = threadIdx.x; w < 2 * nW; w += blockDim.x) m0[w] = 0u;
-  if constexpr (I8)
-    for (int jj = threadIdx.x; jj < prm.nB; jj += blockDim.x) sk_s[jj] = prm.sk[bh * prm.nB + jj];
-  __syncthreads();
   {
-    const int32_t* r0 = prm.idx + (bh * prm.nB + qb0) * (long long)prm.k;
-    const int32_t* r1 = prm.idx + (bh * prm.nB + qb1) * (long long)prm.k;
+    // an id out of range or out of order is reported; out-of-range ids are
+    // replaced by 0 so that no load or scale lookup leaves its tensor
+    const int32_t* r0 = prm.idx + (bh * prm.nB + qb0) * (long long)n;
+    const int32_t* r1 = prm.idx + (bh * prm.nB + (has1 ? qb1 : qb0)) * (long long)n;
     bool bad = false;
-    for (int t = threadIdx.x; t < prm.k; t += blockDim.x) {
-      const int j = r0[t];
-      if (j < 0 || j >= prm.nB || (t > 0 && r0[t - 1] >= j)) bad = true;
-      else atomicOr(&m0[j >> 5], 1u << (j & 31));
-      if (has1) {
-        const int j1 = r1[t];
-        if (j1 < 0 || j1 >= prm.nB || (t > 0 && r1[t - 1] >= j1)) bad = true;
-        else atomicOr(&m1[j1 >> 5], 1u << (j1 & 31));
-      }
+    for (int t = threadIdx.x; t < n; t += blockDim.x) {
+      int j0 = r0[t], j1 = r1[t];
+      if (j0 < 0 || j0 >= prm.nB || (t > 0 && r0[t - 1] >= j0)) bad = true;
+      if (j1 < 0 || j1 >= prm.nB || (t > 0 && r1[t - 1] >= j1)) bad = true;
+      idx0[t] = (j0 < 0 || j0 >= prm.nB) ? 0 : j0;
+      idx1[t] = (j1 < 0 || j1 >= prm.nB) ? 0 : j1;
     }
     if (bad) report_error(-7);
   }
@@ -174,14 +155,6 @@ __global__ void __launch_bounds__(192, I8 ? 2 : 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (warp == 0) {
-    int cnt = 0;
-    for (int w = lane; w < nW; w += 32) cnt += __popc(m0[w] | m1[w]);
-    cnt = __reduce_add_sync(0xffffffffu, cnt);
-    if (lane == 0) n_union = cnt;
-  }
-  __syncthreads();
-  const int n = n_union;
   const uint32_t tbase = tmem_slot;
   const uint32_t sQ = smem_u32(sm + C::OFF_Q);
 
@@ -194,29 +167,45 @@ __global__ void __launch_bounds__(192, I8 ? 2 : 1)
       mbar_arrive_expect_tx(&bar_q, C::Q_BYTES);
       for (int a = 0; a < C::NATOM; ++a)
         tma_load_4d(sm + C::OFF_Q + a * 128 * C::ATOM, &tmQ, &bar_q, a * C::ATOM / C::ESZ, qb0 * kBlock, h_idx, b_idx);
-      UnionWalk uw;
-      uw.init(m0, m1, nW);
-      int j, fl, c = 0;
-      while (uw.next(j, fl)) {
-        const int s = c % C::NSTAGE;
-        if (c >= C::NSTAGE && !mbar_wait(&bar_empty[s], ((c / C::NSTAGE) - 1) & 1, &abort_flag, prm.limit_ns)) {
-          abort_flag = 1;
-          report_error(-6);
-          break;
-        }
-        mbar_arrive_expect_tx(&bar_full[s], 2 * C::KV_BYTES);
+      const uint32_t kv_tx = (has1 ? 2 : 1) * C::KV_BYTES;
+      bool ok = true;
+      int nk = 0, nv = 0;  // K and V block pairs issued so far
+      for (int c = 0; c < n; ++c) {
+        const int ks = c % C::KSTAGE, vs = c % C::VSTAGE;
+        const int j0 = idx0[c], j1 = idx1[c];
+        ok = c < C::KSTAGE || mbar_wait(&bar_kempty[ks], ((c / C::KSTAGE) - 1) & 1, &abort_flag, prm.limit_ns);
+        if (!ok) break;
+        uint8_t* sk = sm + C::OFF_K + ks * 2 * C::KV_BYTES;
+        mbar_arrive_expect_tx(&bar_kfull[ks], kv_tx);
         for (int a = 0; a < C::NATOM; ++a) {
-          tma_load_4d(sm + C::OFF_K + s * C::KV_BYTES + a * 64 * C::ATOM, &tmK, &bar_full[s], a * C::ATOM / C::ESZ,
-                      j * kBlock, h_idx, b_idx);
-          tma_load_4d(sm + C::OFF_V + s * C::KV_BYTES + a * 64 * C::ATOM, &tmV, &bar_full[s], a * C::ATOM / C::ESZ,
-                      j * kBlock, h_idx, b_idx);
+          tma_load_4d(sk + a * 64 * C::ATOM, &tmK, &bar_kfull[ks], a * C::ATOM / C::ESZ, j0 * kBlock, h_idx, b_idx);
+          if (has1)
+            tma_load_4d(sk + C::KV_BYTES + a * 64 * C::ATOM, &tmK, &bar_kfull[ks], a * C::ATOM / C::ESZ, j1 * kBlock,
+                        h_idx, b_idx);
         }
-        ++c;
+        ++nk;
+        ok = c < C::VSTAGE || mbar_wait(&bar_vempty[vs], ((c / C::VSTAGE) - 1) & 1, &abort_flag, prm.limit_ns);
+        if (!ok) break;
+        uint8_t* sv = sm + C::OFF_V + vs * 2 * C::KV_BYTES;
+        mbar_arrive_expect_tx(&bar_vfull[vs], kv_tx);
+        for (int a = 0; a < C::NATOM; ++a) {
+          tma_load_4d(sv + a * 64 * C::ATOM, &tmV, &bar_vfull[vs], a * C::ATOM / C::ESZ, j0 * kBlock, h_idx, b_idx);
+          if (has1)
+            tma_load_4d(sv + C::KV_BYTES + a * 64 * C::ATOM, &tmV, &bar_vfull[vs], a * C::ATOM / C::ESZ, j1 * kBlock,
+                        h_idx, b_idx);
+        }
+        ++nv;
+      }
+      if (!ok) {
+        abort_flag = 1;
+        report_error(-6);
       }
       // drain: every issued load lands before the CTA may exit
       mbar_wait(&bar_q, 0, &never_abort, prm.limit_ns);
-      for (int cc = c - C::NSTAGE < 0 ? 0 : c - C::NSTAGE; cc < c; ++cc)
-        mbar_wait(&bar_full[cc % C::NSTAGE], (cc / C::NSTAGE) & 1, &never_abort, prm.limit_ns);
+      for (int cc = nk - C::KSTAGE < 0 ? 0 : nk - C::KSTAGE; cc < nk; ++cc)
+        mbar_wait(&bar_kfull[cc % C::KSTAGE], (cc / C::KSTAGE) & 1, &never_abort, prm.limit_ns);
+      for (int cc = nv - C::VSTAGE < 0 ? 0 : nv - C::VSTAGE; cc < nv; ++cc)
+        mbar_wait(&bar_vfull[cc % C::VSTAGE], (cc / C::VSTAGE) & 1, &never_abort, prm.limit_ns);
     }
   } else if (warp == 1) {
     // ================= MMA issuer =================
@@ -225,36 +214,51 @@ __global__ void __launch_bounds__(192, I8 ? 2 : 1)
       tc_fence_after();
       for (int c = 0; ok && c <= n; ++c) {
         if (c < n) {
-          const int s = c % C::NSTAGE;
-          ok = mbar_wait(&bar_full[s], (c / C::NSTAGE) & 1, &abort_flag, prm.limit_ns) &&
+          const int ks = c % C::KSTAGE;
+          ok = mbar_wait(&bar_kfull[ks], (c / C::KSTAGE) & 1, &abort_flag, prm.limit_ns) &&
                mbar_wait(&bar_sfree, c & 1, &abort_flag, prm.limit_ns);
           if (!ok) break;
           tc_fence_after();
-          const uint32_t sK = smem_u32(sm + C::OFF_K + s * C::KV_BYTES);
+          const uint32_t sK = smem_u32(sm + C::OFF_K + ks * 2 * C::KV_BYTES);
 #pragma unroll
-          for (int kk = 0; kk < C::ROWB / 32; ++kk) {
-            const int a = (kk * 32) / C::ATOM, off = (kk * 32) % C::ATOM;
-            const uint64_t ad = smem_desc(sQ + a * 128 * C::ATOM + off, 16, 8 * C::ATOM, C::SW_QKV);
-            const uint64_t bd = smem_desc(sK + a * 64 * C::ATOM + off, 16, 8 * C::ATOM, C::SW_QKV);
-            // INT8: accumulate onto the magic-number start the softmax warps wrote
-            mma_ss<I8 ? KIND_I8 : KIND_F16>(tbase + C::S_COL, ad, bd, C::IDESC_S, (I8 || kk > 0) ? 1u : 0u);
+          for (int s = 0; s < 2; ++s) {
+            if (s == 1 && !has1) break;
+#pragma unroll
+            for (int kk = 0; kk < C::ROWB / 32; ++kk) {
+              const int a = (kk * 32) / C::ATOM, off = (kk * 32) % C::ATOM;
+              const uint64_t ad =
+                  smem_desc(sQ + a * 128 * C::ATOM + s * 64 * C::ATOM + off, 16, 8 * C::ATOM, C::SW_QKV);
+              const uint64_t bd = smem_desc(sK + s * C::KV_BYTES + a * 64 * C::ATOM + off, 16, 8 * C::ATOM, C::SW_QKV);
+              // INT8: accumulate onto the magic-number start the softmax warps wrote
+              mma_ss<I8 ? KIND_I8 : KIND_F16>(tbase + s * C::LANE_B + C::S_COL, ad, bd, C::IDESC_S,
+                                              (I8 || kk > 0) ? 1u : 0u);
+            }
           }
           mma_commit(&bar_sfull);
+          mma_commit(&bar_kempty[ks]);
         }
         if (c >= 1) {
-          const int cp = c - 1, s = cp % C::NSTAGE, pb = cp & 1;
-          ok = mbar_wait(&bar_pfull[pb], (cp >> 1) & 1, &abort_flag, prm.limit_ns);
+          const int cp = c - 1, vs = cp % C::VSTAGE;
+          ok = mbar_wait(&bar_vfull[vs], (cp / C::VSTAGE) & 1, &abort_flag, prm.limit_ns) &&
+               mbar_wait(&bar_pfull, cp & 1, &abort_flag, prm.limit_ns);
           if (!ok) break;
           tc_fence_after();
-          const uint32_t sV = smem_u32(sm + C::OFF_V + s * C::KV_BYTES);
+          const uint32_t sV = smem_u32(sm + C::OFF_V + vs * 2 * C::KV_BYTES);
+          const uint32_t sP = smem_u32(sm + C::OFF_P);
 #pragma unroll
-          for (int kk = 0; kk < 64 / C::KEYS_PER_MMA; ++kk) {
-            const uint64_t bd = smem_desc(sV + kk * C::KEYS_PER_MMA * C::ATOM, 64 * C::ATOM, 8 * C::ATOM, C::SW_QKV);
-            mma_ts<I8 ? KIND_F8F6F4 : KIND_F16>(tbase + C::O_COL, tbase + C::P_COL + pb * C::P_COLS + kk * 8, bd,
-                                                C::IDESC_PV, (cp > 0 || kk > 0) ? 1u : 0u);
+          for (int s = 0; s < 2; ++s) {
+            if (s == 1 && !has1) break;
+#pragma unroll
+            for (int kk = 0; kk < 64 / C::KEYS_PER_MMA; ++kk) {
+              const uint64_t ad = smem_desc(sP + s * C::P_BYTES + kk * 32, 16, 8 * C::P_ROWB, C::SW_P);
+              const uint64_t bd = smem_desc(sV + s * C::KV_BYTES + kk * C::KEYS_PER_MMA * C::ATOM, 64 * C::ATOM,
+                                            8 * C::ATOM, C::SW_QKV);
+              mma_ss<I8 ? KIND_F8F6F4 : KIND_F16>(tbase + s * C::LANE_B + C::O_COL, ad, bd, C::IDESC_PV,
+                                                  (cp > 0 || kk > 0) ? 1u : 0u);
+            }
           }
           mma_commit(&bar_odone);
-          mma_commit(&bar_empty[s]);
+          mma_commit(&bar_vempty[vs]);
         }
       }
       if (!ok) {
@@ -268,15 +272,20 @@ __global__ void __launch_bounds__(192, I8 ? 2 : 1)
   } else {
     // ================= softmax / correction / epilogue =================
     const int quarter = warp & 3;
-    const int r = quarter * 32 + lane;           // tile row == TMEM lane
-    const int half = r >> 6;
-    const int qblk = half ? qb1 : qb0;
-    const int t = qblk * kBlock + (r & 63);      // token index of this row
+    const int stream = lane >> 4;
+    const int row = quarter * 16 + (lane & 15);   // row within this stream's query block
+    const int qblk = stream ? qb1 : qb0;
+    const bool valid = stream == 0 || has1;
+    const int t = qblk * kBlock + row;            // token index of this row
     const uint32_t lane_addr = tbase + ((uint32_t)(quarter * 32) << 16);
+    const int32_t* my_idx = stream ? idx1 : idx0;
+    const float* sk_row = prm.sk + bh * prm.nB;
     float sq = 1.0f;
     if constexpr (I8) sq = prm.sq[bh * prm.nB + min(qblk, prm.nB - 1)];
     float m_run = -INFINITY, l_run = 0.f;
-    // the S tile starts free (INT8: at the magic-number start value)
+    // this thread's row of its stream's P tile (K-major, swizzled)
+    uint8_t* prow = sm + C::OFF_P + stream * C::P_BYTES;
+    // the S columns start free (INT8: at the magic-number start value)
     if constexpr (I8) {
       uint32_t mg[32];
 #pragma unroll
@@ -287,13 +296,16 @@ __global__ void __launch_bounds__(192, I8 ? 2 : 1)
     }
     tc_fence_before();
     mbar_arrive(&bar_sfree);
-    UnionWalk uw;
-    uw.init(m0, m1, nW);
     bool ok = true;
-    int j = 0, fl = 0;
+    int j_next = n > 0 ? my_idx[0] : 0;
+    float sk_next = (I8 && n > 0) ? __ldg(sk_row + j_next) : 1.f;
     for (int c = 0; c < n; ++c) {
-      uw.next(j, fl);
-      const int bsel = c & 1;
+      const int j = j_next;
+      const float skj = sk_next;
+      if (c + 1 < n) {  // the next step's block and K scale, fetched a step ahead
+        j_next = my_idx[c + 1];
+        if constexpr (I8) sk_next = __ldg(sk_row + j_next);
+      }
       ok = mbar_wait(&bar_sfull, c & 1, &abort_flag, prm.limit_ns);
       if (!ok) break;
       tc_fence_after();
@@ -305,8 +317,8 @@ __global__ void __launch_bounds__(192, I8 ? 2 : 1)
         tmem_ld32(lane_addr + C::S_COL + 32, hi);
         tmem_wait_ld();
       }
-      // hand the S tile back at once (INT8: restarted at the magic value) so the
-      // next S = QK^T runs on the tensor core while this block's softmax runs
+      // hand the S columns back at once (INT8: restarted at the magic value) so
+      // the next S = QK^T runs on the tensor core while this block's softmax runs
       if constexpr (I8) {
         uint32_t mg[32];
 #pragma unroll
@@ -317,14 +329,13 @@ __global__ void __launch_bounds__(192, I8 ? 2 : 1)
       }
       tc_fence_before();
       mbar_arrive(&bar_sfree);
-      const bool use = ((fl >> half) & 1) != 0;
       const int nvalid = (j == prm.nB - 1) ? (prm.L - j * kBlock) : kBlock;
       float sc = prm.scale_log2;
-      if constexpr (I8) sc *= sq * sk_s[j];
+      if constexpr (I8) sc *= sq * skj;
       float m_new = m_run, alpha = 1.f, psum = 0.f;
-      constexpr int PW = C::P_COLS;
+      constexpr int PW = C::P_ROWB / 4;
       uint32_t pk[PW];
-      if (use) {
+      if (valid) {
         // block max (scores read as floats; INT8 ones carry the magic offset)
         float mx;
         if (nvalid == kBlock) {
@@ -388,12 +399,12 @@ __global__ void __launch_bounds__(192, I8 ? 2 : 1)
         for (int i = 0; i < PW; ++i) pk[i] = 0u;
       }
       if (c >= 1) {
-        // PV of the previous block is complete: O may be rescaled and the P
-        // buffer of block c-2 is free again
+        // the previous block's P.V is complete: O may be rescaled and the P
+        // tiles may be overwritten
         ok = mbar_wait(&bar_odone, (c - 1) & 1, &abort_flag, prm.limit_ns);
         if (!ok) break;
         tc_fence_after();
-        const bool need_rescale = use && m_run != -INFINITY && m_new > m_run;
+        const bool need_rescale = valid && m_run != -INFINITY && m_new > m_run;
         if (__any_sync(0xffffffffu, need_rescale)) {
           const float f = need_rescale ? alpha : 1.f;
 #pragma unroll
@@ -405,18 +416,18 @@ __global__ void __launch_bounds__(192, I8 ? 2 : 1)
             for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * f);
             tmem_st32(lane_addr + C::O_COL + cc, o);
           }
+          tmem_wait_st();
         }
       }
-      // P of this block into its TMEM buffer: the A operand of PV
-      if constexpr (I8) {
-        tmem_st16(lane_addr + C::P_COL + bsel * C::P_COLS, pk);
-      } else {
-        tmem_st32(lane_addr + C::P_COL + bsel * C::P_COLS, *reinterpret_cast<uint32_t(*)[32]>(pk));
-      }
-      tmem_wait_st();
+      // P row into shared memory: the A operand of this stream's P.V
+#pragma unroll
+      for (int ch = 0; ch < C::P_ROWB / 16; ++ch)
+        *reinterpret_cast<uint4*>(prow + swz_offset(row, ch, C::P_ROWB)) =
+            make_uint4(pk[4 * ch], pk[4 * ch + 1], pk[4 * ch + 2], pk[4 * ch + 3]);
+      fence_proxy_async_smem();
       tc_fence_before();
-      mbar_arrive(&bar_pfull[bsel]);
-      if (use) {
+      mbar_arrive(&bar_pfull);
+      if (valid) {
         l_run = l_run * alpha + psum;
         m_run = m_new;
       }
@@ -425,14 +436,14 @@ __global__ void __launch_bounds__(192, I8 ? 2 : 1)
       abort_flag = 1;
       report_error(-6);
     } else {
-      // epilogue: wait for the last PV, normalise, store bf16 rows
+      // epilogue: wait for the last P.V, normalise, store bf16 rows
       ok = n == 0 || mbar_wait(&bar_odone, (n - 1) & 1, &abort_flag, prm.limit_ns);
       if (!ok) {
         abort_flag = 1;
         report_error(-6);
       } else {
         tc_fence_after();
-        const bool store = t < prm.L && (half == 0 || has1) && l_run > 0.f;
+        const bool store = valid && t < prm.L && l_run > 0.f;
         const float inv_l = store ? 1.0f / l_run : 0.f;
         __nv_bfloat16* orow = prm.o + (long long)b_idx * prm.osB + (long long)h_idx * prm.osH + (long long)t * prm.osL;
 #pragma unroll

@@ -140,8 +140,7 @@ lx_status launch_attn(const CUtensorMap& mq, const CUtensorMap& mk, const CUtens
                       const lx_bhld* O, const float* qs, const float* ks, const float* vs, cudaStream_t s) {
   using C = lx::AttnCfg<D, I8>;
   const int64_t nB = plan->nB;
-  const int nW = (int)((nB + 31) / 32);
-  const size_t smem = 1024 + C::OFF_MASK + 2 * sizeof(uint32_t) * nW + (I8 ? sizeof(float) * nB : 0);
+  const size_t smem = 1024 + C::OFF_IDX + 2 * sizeof(int32_t) * (size_t)plan->k;
   if (smem > 227 * 1024) return LX_ERR_UNSUPPORTED;
   if (cudaFuncSetAttribute(lx::sparse_attn_kernel<D, I8>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
       cudaSuccess)
