@@ -210,6 +210,13 @@ __global__ void __launch_bounds__(192, I8 ? 2 : 1)
   } else if (warp == 1) {
     // ================= MMA issuer =================
     if (lane == 0) {
+      // Descriptors of stage 0 / stream A; a shared-memory descriptor's start
+      // address sits in its low 14 bits (address >> 4, below 256 KB), so other
+      // stages, streams and K steps are plain additions of (offset >> 4).
+      const uint64_t dQ = smem_desc(sQ, 16, 8 * C::ATOM, C::SW_QKV);
+      const uint64_t dK = smem_desc(smem_u32(sm + C::OFF_K), 16, 8 * C::ATOM, C::SW_QKV);
+      const uint64_t dP = smem_desc(smem_u32(sm + C::OFF_P), 16, 8 * C::P_ROWB, C::SW_P);
+      const uint64_t dV = smem_desc(smem_u32(sm + C::OFF_V), 64 * C::ATOM, 8 * C::ATOM, C::SW_QKV);
       bool ok = mbar_wait(&bar_q, 0, &abort_flag, prm.limit_ns);
       tc_fence_after();
       for (int c = 0; ok && c <= n; ++c) {
@@ -219,16 +226,15 @@ __global__ void __launch_bounds__(192, I8 ? 2 : 1)
                mbar_wait(&bar_sfree, c & 1, &abort_flag, prm.limit_ns);
           if (!ok) break;
           tc_fence_after();
-          const uint32_t sK = smem_u32(sm + C::OFF_K + ks * 2 * C::KV_BYTES);
+          const uint64_t dKs = dK + (uint64_t)((ks * 2 * C::KV_BYTES) >> 4);
 #pragma unroll
           for (int s = 0; s < 2; ++s) {
             if (s == 1 && !has1) break;
 #pragma unroll
             for (int kk = 0; kk < C::ROWB / 32; ++kk) {
               const int a = (kk * 32) / C::ATOM, off = (kk * 32) % C::ATOM;
-              const uint64_t ad =
-                  smem_desc(sQ + a * 128 * C::ATOM + s * 64 * C::ATOM + off, 16, 8 * C::ATOM, C::SW_QKV);
-              const uint64_t bd = smem_desc(sK + s * C::KV_BYTES + a * 64 * C::ATOM + off, 16, 8 * C::ATOM, C::SW_QKV);
+              const uint64_t ad = dQ + (uint64_t)((a * 128 * C::ATOM + s * 64 * C::ATOM + off) >> 4);
+              const uint64_t bd = dKs + (uint64_t)((s * C::KV_BYTES + a * 64 * C::ATOM + off) >> 4);
               // INT8: accumulate onto the magic-number start the softmax warps wrote
               mma_ss<I8 ? KIND_I8 : KIND_F16>(tbase + s * C::LANE_B + C::S_COL, ad, bd, C::IDESC_S,
                                               (I8 || kk > 0) ? 1u : 0u);
@@ -243,16 +249,14 @@ __global__ void __launch_bounds__(192, I8 ? 2 : 1)
                mbar_wait(&bar_pfull, cp & 1, &abort_flag, prm.limit_ns);
           if (!ok) break;
           tc_fence_after();
-          const uint32_t sV = smem_u32(sm + C::OFF_V + vs * 2 * C::KV_BYTES);
-          const uint32_t sP = smem_u32(sm + C::OFF_P);
+          const uint64_t dVs = dV + (uint64_t)((vs * 2 * C::KV_BYTES) >> 4);
 #pragma unroll
           for (int s = 0; s < 2; ++s) {
             if (s == 1 && !has1) break;
 #pragma unroll
             for (int kk = 0; kk < 64 / C::KEYS_PER_MMA; ++kk) {
-              const uint64_t ad = smem_desc(sP + s * C::P_BYTES + kk * 32, 16, 8 * C::P_ROWB, C::SW_P);
-              const uint64_t bd = smem_desc(sV + s * C::KV_BYTES + kk * C::KEYS_PER_MMA * C::ATOM, 64 * C::ATOM,
-                                            8 * C::ATOM, C::SW_QKV);
+              const uint64_t ad = dP + (uint64_t)((s * C::P_BYTES + kk * 32) >> 4);
+              const uint64_t bd = dVs + (uint64_t)((s * C::KV_BYTES + kk * C::KEYS_PER_MMA * C::ATOM) >> 4);
               mma_ss<I8 ? KIND_F8F6F4 : KIND_F16>(tbase + s * C::LANE_B + C::O_COL, ad, bd, C::IDESC_PV,
                                                   (cp > 0 || kk > 0) ? 1u : 0u);
             }
@@ -339,12 +343,17 @@ __global__ void __launch_bounds__(192, I8 ? 2 : 1)
         // block max (scores read as floats; INT8 ones carry the magic offset)
         float mx;
         if (nvalid == kBlock) {
+          // eight chains of three-input maxima, then a three-level fold
+          const float* f = reinterpret_cast<const float*>(sv);
           float t8[8];
 #pragma unroll
-          for (int i = 0; i < 8; ++i) t8[i] = __uint_as_float(sv[i]);
-#pragma unroll
-          for (int u = 8; u < 64; ++u) t8[u & 7] = fmaxf(t8[u & 7], __uint_as_float(sv[u]));
-          mx = fmaxf(fmaxf(fmaxf(t8[0], t8[1]), fmaxf(t8[2], t8[3])), fmaxf(fmaxf(t8[4], t8[5]), fmaxf(t8[6], t8[7])));
+          for (int i = 0; i < 8; ++i) {
+            float a = fmax3(f[i], f[i + 8], f[i + 16]);
+            a = fmax3(a, f[i + 24], f[i + 32]);
+            a = fmax3(a, f[i + 40], f[i + 48]);
+            t8[i] = fmaxf(a, f[i + 56]);
+          }
+          mx = fmaxf(fmax3(t8[0], t8[1], t8[2]), fmax3(t8[3], t8[4], fmax3(t8[5], t8[6], t8[7])));
         } else {
           mx = -INFINITY;
 #pragma unroll
@@ -380,9 +389,8 @@ __global__ void __launch_bounds__(192, I8 ? 2 : 1)
           const float p0 = __uint_as_float(sv[u]), p1 = __uint_as_float(sv[u + 1]);
           acc2[(u >> 1) & 3] = add2(acc2[(u >> 1) & 3], f2pack(p0, p1));
           if constexpr (I8) {
-            const uint32_t e = e4m3x2(p0, p1);
-            if ((u & 2) == 0) pk[u >> 2] = e;
-            else pk[u >> 2] |= e << 16;
+            if ((u & 2) == 0)
+              pk[u >> 2] = e4m3x4(p0, p1, __uint_as_float(sv[u + 2]), __uint_as_float(sv[u + 3]));
           } else {
             __nv_bfloat162 hb = __floats2bfloat162_rn(p0, p1);
             pk[u >> 1] = *reinterpret_cast<uint32_t*>(&hb);
@@ -407,13 +415,19 @@ __global__ void __launch_bounds__(192, I8 ? 2 : 1)
         const bool need_rescale = valid && m_run != -INFINITY && m_new > m_run;
         if (__any_sync(0xffffffffu, need_rescale)) {
           const float f = need_rescale ? alpha : 1.f;
+          const uint64_t f2 = f2pack(f, f);
 #pragma unroll
           for (int cc = 0; cc < D; cc += 32) {
             uint32_t o[32];
             tmem_ld32(lane_addr + C::O_COL + cc, o);
             tmem_wait_ld();
 #pragma unroll
-            for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * f);
+            for (int i = 0; i < 32; i += 2) {
+              float a, b;
+              f2unpack(mul2(f2pack(__uint_as_float(o[i]), __uint_as_float(o[i + 1])), f2), a, b);
+              o[i] = __float_as_uint(a);
+              o[i + 1] = __float_as_uint(b);
+            }
             tmem_st32(lane_addr + C::O_COL + cc, o);
           }
           tmem_wait_st();

@@ -31,6 +31,14 @@ __device__ __forceinline__ uint32_t e4m3x2(float lo, float hi) {
   asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
   return (uint32_t)r;
 }
+// four floats to four E4M3 bytes, a in the lowest byte
+__device__ __forceinline__ uint32_t e4m3x4(float a, float b, float c, float d) {
+  uint32_t r;
+  asm("{\n .reg .b16 lo, hi;\n cvt.rn.satfinite.e4m3x2.f32 lo, %2, %1;\n"
+      " cvt.rn.satfinite.e4m3x2.f32 hi, %4, %3;\n mov.b32 %0, {lo, hi};\n}"
+      : "=r"(r) : "f"(a), "f"(b), "f"(c), "f"(d));
+  return r;
+}
 
 // ---------------------------------------------------------------------------
 // Q/K: one 128-thread CTA per (tensor, b*h, block).  Thread t covers row t/2,
