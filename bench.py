@@ -33,7 +33,7 @@ METRIC = "block-sparse attn effective TFLOPS (720p grid, 40x128, keep 10%)"
 # kernel build: the ncu capture in profiles/attn_int8fp8_720p_8heads_ncu.md
 # (8 of the 40 heads; traffic grows with the head count, so x5).  Set to None
 # whenever the attention kernel changes until it is captured again.
-ATTN_DRAM_BYTES_PER_LAUNCH = 5 * (238.465280e6 + 125.838336e6)
+ATTN_DRAM_BYTES_PER_LAUNCH = None
 
 
 def reduce_max(x: float, device) -> float:

@@ -15,10 +15,14 @@
 // half-subpartition layout of an M=64 tcgen05 accumulator), so one warp's
 // 32x32b TMEM load returns 16 rows of A and 16 rows of B.
 //
-// Roles (6 warps): warp 0 = TMA producer (Q once; K blocks of both streams
-// into a 3-stage ring, V blocks into a 2-stage ring); warp 1 = TMEM allocator
-// + MMA issuer (S_A, S_B = Q K^T into the S columns, then O_A, O_B += P V into
-// the O columns, P and V read from shared memory); warps 2..5 = softmax /
+// S is computed for two consecutive kept blocks of a stream at once (M=64,
+// N=128 over the stacked blocks); P.V and the O rescale stay per 64-key block.
+//
+// Roles (6 warps): warp 0 = TMA producer (Q once; K blocks of both streams, a
+// pair of steps at a time, into one stage; V blocks into a 2-stage ring);
+// warp 1 = TMEM allocator + MMA issuer (S_A, S_B = Q K^T into the S columns,
+// then O_A, O_B += P V into the O columns, P and V read from shared memory);
+// warps 2..5 = softmax /
 // correction / epilogue, one thread per (stream, row): thread t of warp w
 // reads TMEM lane 32*(w%4) + t, i.e. row 16*(w%4) + t%16 of stream t/16.
 //
@@ -43,7 +47,7 @@ struct AttnCfg {
   static constexpr int NATOM = ROWB / ATOM;               // atom columns per row
   static constexpr int Q_BYTES = 128 * ROWB;              // rows 0-63: stream A, rows 64-127: stream B
   static constexpr int KV_BYTES = 64 * ROWB;              // one K (or V) block
-  static constexpr int KSTAGE = 3;                        // K ring (A and B blocks per stage)
+  static constexpr int KPAIR_BYTES = 2 * KV_BYTES;        // one stream's two K blocks: [NATOM][128 rows][ATOM]
   static constexpr int VSTAGE = 2;                        // V ring (A and B blocks per stage)
   static constexpr int P_ROWB = 64 * ESZ;                 // P row: 64 keys
   static constexpr int P_BYTES = 64 * P_ROWB;             // P of one stream, K-major, swizzled
@@ -51,15 +55,15 @@ struct AttnCfg {
   static constexpr uint32_t SW_P = P_ROWB == 128 ? SW_128B : SW_64B;
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_K = OFF_Q + Q_BYTES;
-  static constexpr int OFF_V = OFF_K + KSTAGE * 2 * KV_BYTES;
+  static constexpr int OFF_V = OFF_K + 2 * KPAIR_BYTES;
   static constexpr int OFF_P = OFF_V + VSTAGE * 2 * KV_BYTES;
   static constexpr int OFF_IDX = OFF_P + 2 * P_BYTES;     // the two kept lists (2 x k int32) follow
-  static constexpr int S_COL = 0;                         // TMEM: S, cols [0, 64)
+  static constexpr int S_COL = 0;                         // TMEM: S of a step pair, cols [0, 128)
   static constexpr int O_COL = 128;                       // TMEM: O accumulator, D cols
   static constexpr uint32_t LANE_B = 16u << 16;           // TMEM address offset of stream B (lane 16)
   static constexpr uint32_t TMEM_COLS = 256;
   static constexpr uint32_t IDESC_S =
-      instr_desc(I8 ? IDESC_DS32 : IDESC_DF32, I8 ? IDESC_S8 : IDESC_BF16, I8 ? IDESC_S8 : IDESC_BF16, 0, 0, 64, 64);
+      instr_desc(I8 ? IDESC_DS32 : IDESC_DF32, I8 ? IDESC_S8 : IDESC_BF16, I8 ? IDESC_S8 : IDESC_BF16, 0, 0, 64, 128);
   static constexpr uint32_t IDESC_PV =
       instr_desc(IDESC_DF32, I8 ? IDESC_E4M3 : IDESC_BF16, I8 ? IDESC_E4M3 : IDESC_BF16, 0, 1, 64, D);
   static constexpr int KEYS_PER_MMA = 32 / ESZ;           // 32 bytes of K per instruction
@@ -97,7 +101,7 @@ __global__ void __launch_bounds__(192, I8 ? 2 : 1)
   using C = AttnCfg<D, I8>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  __shared__ uint64_t bar_q, bar_kfull[C::KSTAGE], bar_kempty[C::KSTAGE], bar_vfull[C::VSTAGE],
+  __shared__ uint64_t bar_q, bar_kfull, bar_kempty, bar_vfull[C::VSTAGE],
       bar_vempty[C::VSTAGE], bar_sfull, bar_sfree, bar_pfull, bar_odone, bar_drain;
   __shared__ uint32_t tmem_slot;
   __shared__ volatile int abort_flag;
@@ -110,16 +114,15 @@ __global__ void __launch_bounds__(192, I8 ? 2 : 1)
   const int qb0 = 2 * pair, qb1 = 2 * pair + 1;
   const bool has1 = qb1 < prm.nB;
   const int n = prm.k;  // steps: every stream walks exactly k kept blocks
+  const int npairs = (n + 1) >> 1;  // S is computed for steps 2p and 2p+1 together
   int32_t* idx0 = reinterpret_cast<int32_t*>(sm + C::OFF_IDX);
   int32_t* idx1 = idx0 + n;
 
   // ---- prologue: barriers, the two kept lists (validated), TMEM
   if (threadIdx.x == 0) {
     mbar_init(&bar_q, 1);
-    for (int s = 0; s < C::KSTAGE; ++s) {
-      mbar_init(&bar_kfull[s], 1);
-      mbar_init(&bar_kempty[s], 1);
-    }
+    mbar_init(&bar_kfull, 1);
+    mbar_init(&bar_kempty, 1);
     for (int s = 0; s < C::VSTAGE; ++s) {
       mbar_init(&bar_vfull[s], 1);
       mbar_init(&bar_vempty[s], 1);
@@ -169,30 +172,36 @@ __global__ void __launch_bounds__(192, I8 ? 2 : 1)
         tma_load_4d(sm + C::OFF_Q + a * 128 * C::ATOM, &tmQ, &bar_q, a * C::ATOM / C::ESZ, qb0 * kBlock, h_idx, b_idx);
       const uint32_t kv_tx = (has1 ? 2 : 1) * C::KV_BYTES;
       bool ok = true;
-      int nk = 0, nv = 0;  // K and V block pairs issued so far
+      int nk = 0, nv = 0;  // K pairs and V steps issued so far
       for (int c = 0; c < n; ++c) {
-        const int ks = c % C::KSTAGE, vs = c % C::VSTAGE;
-        const int j0 = idx0[c], j1 = idx1[c];
-        ok = c < C::KSTAGE || mbar_wait(&bar_kempty[ks], ((c / C::KSTAGE) - 1) & 1, &abort_flag, prm.limit_ns);
-        if (!ok) break;
-        uint8_t* sk = sm + C::OFF_K + ks * 2 * C::KV_BYTES;
-        mbar_arrive_expect_tx(&bar_kfull[ks], kv_tx);
-        for (int a = 0; a < C::NATOM; ++a) {
-          tma_load_4d(sk + a * 64 * C::ATOM, &tmK, &bar_kfull[ks], a * C::ATOM / C::ESZ, j0 * kBlock, h_idx, b_idx);
-          if (has1)
-            tma_load_4d(sk + C::KV_BYTES + a * 64 * C::ATOM, &tmK, &bar_kfull[ks], a * C::ATOM / C::ESZ, j1 * kBlock,
-                        h_idx, b_idx);
+        if ((c & 1) == 0) {
+          // K blocks of steps c and c+1 (both streams) into the pair stage,
+          // once S of the previous pair has read it
+          const int p = c >> 1;
+          ok = p == 0 || mbar_wait(&bar_kempty, (p - 1) & 1, &abort_flag, prm.limit_ns);
+          if (!ok) break;
+          const int nb = (c + 1 < n) ? 2 : 1;
+          mbar_arrive_expect_tx(&bar_kfull, (uint32_t)nb * kv_tx);
+          for (int s = 0; s < (has1 ? 2 : 1); ++s) {
+            const int32_t* ids = s ? idx1 : idx0;
+            for (int b = 0; b < nb; ++b)
+              for (int a = 0; a < C::NATOM; ++a)
+                tma_load_4d(sm + C::OFF_K + s * C::KPAIR_BYTES + a * 128 * C::ATOM + b * 64 * C::ATOM, &tmK,
+                            &bar_kfull, a * C::ATOM / C::ESZ, ids[c + b] * kBlock, h_idx, b_idx);
+          }
+          ++nk;
         }
-        ++nk;
+        const int vs = c % C::VSTAGE;
         ok = c < C::VSTAGE || mbar_wait(&bar_vempty[vs], ((c / C::VSTAGE) - 1) & 1, &abort_flag, prm.limit_ns);
         if (!ok) break;
+        const int j0 = idx0[c], j1 = idx1[c];
         uint8_t* sv = sm + C::OFF_V + vs * 2 * C::KV_BYTES;
         mbar_arrive_expect_tx(&bar_vfull[vs], kv_tx);
         for (int a = 0; a < C::NATOM; ++a) {
           tma_load_4d(sv + a * 64 * C::ATOM, &tmV, &bar_vfull[vs], a * C::ATOM / C::ESZ, j0 * kBlock, h_idx, b_idx);
           if (has1)
-            tma_load_4d(sv + C::KV_BYTES + a * 64 * C::ATOM, &tmV, &bar_vfull[vs], a * C::ATOM / C::ESZ, j1 * kBlock,
-                        h_idx, b_idx);
+            tma_load_4d(sv + C::KV_BYTES + a * 64 * C::ATOM, &tmV, &bar_vfull[vs], a * C::ATOM / C::ESZ,
+                        j1 * kBlock, h_idx, b_idx);
         }
         ++nv;
       }
@@ -202,8 +211,7 @@ __global__ void __launch_bounds__(192, I8 ? 2 : 1)
       }
       // drain: every issued load lands before the CTA may exit
       mbar_wait(&bar_q, 0, &never_abort, prm.limit_ns);
-      for (int cc = nk - C::KSTAGE < 0 ? 0 : nk - C::KSTAGE; cc < nk; ++cc)
-        mbar_wait(&bar_kfull[cc % C::KSTAGE], (cc / C::KSTAGE) & 1, &never_abort, prm.limit_ns);
+      if (nk > 0) mbar_wait(&bar_kfull, (nk - 1) & 1, &never_abort, prm.limit_ns);
       for (int cc = nv - C::VSTAGE < 0 ? 0 : nv - C::VSTAGE; cc < nv; ++cc)
         mbar_wait(&bar_vfull[cc % C::VSTAGE], (cc / C::VSTAGE) & 1, &never_abort, prm.limit_ns);
     }
@@ -219,14 +227,16 @@ __global__ void __launch_bounds__(192, I8 ? 2 : 1)
       const uint64_t dV = smem_desc(smem_u32(sm + C::OFF_V), 64 * C::ATOM, 8 * C::ATOM, C::SW_QKV);
       bool ok = mbar_wait(&bar_q, 0, &abort_flag, prm.limit_ns);
       tc_fence_after();
-      for (int c = 0; ok && c <= n; ++c) {
-        if (c < n) {
-          const int ks = c % C::KSTAGE;
-          ok = mbar_wait(&bar_kfull[ks], (c / C::KSTAGE) & 1, &abort_flag, prm.limit_ns) &&
-               mbar_wait(&bar_sfree, c & 1, &abort_flag, prm.limit_ns);
+      // Iteration c issues S of pair p+1 (when c = 2p+1; pair 0 goes first)
+      // and then P(c).V.  S of pair p+1 needs the softmax to have read both
+      // halves of pair p's S, which it does at the start of step 2p+1.
+      for (int c = -1; ok && c < n; ++c) {
+        const int p = (c + 1) >> 1;  // the pair whose S is issued in this iteration
+        if ((c & 1) != 0 && p < npairs) {  // c = -1, 1, 3, ...
+          ok = mbar_wait(&bar_kfull, p & 1, &abort_flag, prm.limit_ns) &&
+               mbar_wait(&bar_sfree, p & 1, &abort_flag, prm.limit_ns);
           if (!ok) break;
           tc_fence_after();
-          const uint64_t dKs = dK + (uint64_t)((ks * 2 * C::KV_BYTES) >> 4);
 #pragma unroll
           for (int s = 0; s < 2; ++s) {
             if (s == 1 && !has1) break;
@@ -234,19 +244,19 @@ __global__ void __launch_bounds__(192, I8 ? 2 : 1)
             for (int kk = 0; kk < C::ROWB / 32; ++kk) {
               const int a = (kk * 32) / C::ATOM, off = (kk * 32) % C::ATOM;
               const uint64_t ad = dQ + (uint64_t)((a * 128 * C::ATOM + s * 64 * C::ATOM + off) >> 4);
-              const uint64_t bd = dKs + (uint64_t)((s * C::KV_BYTES + a * 64 * C::ATOM + off) >> 4);
+              const uint64_t bd = dK + (uint64_t)((s * C::KPAIR_BYTES + a * 128 * C::ATOM + off) >> 4);
               // INT8: accumulate onto the magic-number start the softmax warps wrote
               mma_ss<I8 ? KIND_I8 : KIND_F16>(tbase + s * C::LANE_B + C::S_COL, ad, bd, C::IDESC_S,
                                               (I8 || kk > 0) ? 1u : 0u);
             }
           }
           mma_commit(&bar_sfull);
-          mma_commit(&bar_kempty[ks]);
+          mma_commit(&bar_kempty);
         }
-        if (c >= 1) {
-          const int cp = c - 1, vs = cp % C::VSTAGE;
-          ok = mbar_wait(&bar_vfull[vs], (cp / C::VSTAGE) & 1, &abort_flag, prm.limit_ns) &&
-               mbar_wait(&bar_pfull, cp & 1, &abort_flag, prm.limit_ns);
+        if (c >= 0) {
+          const int vs = c % C::VSTAGE;
+          ok = mbar_wait(&bar_vfull[vs], (c / C::VSTAGE) & 1, &abort_flag, prm.limit_ns) &&
+               mbar_wait(&bar_pfull, c & 1, &abort_flag, prm.limit_ns);
           if (!ok) break;
           tc_fence_after();
           const uint64_t dVs = dV + (uint64_t)((vs * 2 * C::KV_BYTES) >> 4);
@@ -258,7 +268,7 @@ __global__ void __launch_bounds__(192, I8 ? 2 : 1)
               const uint64_t ad = dP + (uint64_t)((s * C::P_BYTES + kk * 32) >> 4);
               const uint64_t bd = dVs + (uint64_t)((s * C::KV_BYTES + kk * C::KEYS_PER_MMA * C::ATOM) >> 4);
               mma_ss<I8 ? KIND_F8F6F4 : KIND_F16>(tbase + s * C::LANE_B + C::O_COL, ad, bd, C::IDESC_PV,
-                                                  (cp > 0 || kk > 0) ? 1u : 0u);
+                                                  (c > 0 || kk > 0) ? 1u : 0u);
             }
           }
           mma_commit(&bar_odone);
@@ -294,8 +304,8 @@ __global__ void __launch_bounds__(192, I8 ? 2 : 1)
       uint32_t mg[32];
 #pragma unroll
       for (int i = 0; i < 32; ++i) mg[i] = kMagicBits;
-      tmem_st32(lane_addr + C::S_COL, mg);
-      tmem_st32(lane_addr + C::S_COL + 32, mg);
+#pragma unroll
+      for (int q = 0; q < 4; ++q) tmem_st32(lane_addr + C::S_COL + 32 * q, mg);
       tmem_wait_st();
     }
     tc_fence_before();
@@ -310,29 +320,36 @@ __global__ void __launch_bounds__(192, I8 ? 2 : 1)
         j_next = my_idx[c + 1];
         if constexpr (I8) sk_next = __ldg(sk_row + j_next);
       }
-      ok = mbar_wait(&bar_sfull, c & 1, &abort_flag, prm.limit_ns);
-      if (!ok) break;
+      const int half = c & 1;  // which 64 columns of the pair's S
+      const uint32_t s_addr = lane_addr + C::S_COL + 64 * half;
+      if (half == 0) {
+        ok = mbar_wait(&bar_sfull, (c >> 1) & 1, &abort_flag, prm.limit_ns);
+        if (!ok) break;
+      }
       tc_fence_after();
       uint32_t sv[64];
       {
         uint32_t (&lo)[32] = *reinterpret_cast<uint32_t(*)[32]>(&sv[0]);
         uint32_t (&hi)[32] = *reinterpret_cast<uint32_t(*)[32]>(&sv[32]);
-        tmem_ld32(lane_addr + C::S_COL, lo);
-        tmem_ld32(lane_addr + C::S_COL + 32, hi);
+        tmem_ld32(s_addr, lo);
+        tmem_ld32(s_addr + 32, hi);
         tmem_wait_ld();
       }
-      // hand the S columns back at once (INT8: restarted at the magic value) so
-      // the next S = QK^T runs on the tensor core while this block's softmax runs
+      // INT8: restart these columns at the magic value; after the second half
+      // of the pair the S columns go back to the MMA thread at once, so the
+      // next pair's S = QK^T runs while this block's softmax runs
       if constexpr (I8) {
         uint32_t mg[32];
 #pragma unroll
         for (int i = 0; i < 32; ++i) mg[i] = kMagicBits;
-        tmem_st32(lane_addr + C::S_COL, mg);
-        tmem_st32(lane_addr + C::S_COL + 32, mg);
+        tmem_st32(s_addr, mg);
+        tmem_st32(s_addr + 32, mg);
         tmem_wait_st();
       }
-      tc_fence_before();
-      mbar_arrive(&bar_sfree);
+      if (half == 1) {
+        tc_fence_before();
+        mbar_arrive(&bar_sfree);
+      }
       const int nvalid = (j == prm.nB - 1) ? (prm.L - j * kBlock) : kBlock;
       float sc = prm.scale_log2;
       if constexpr (I8) sc *= sq * skj;
