@@ -54,6 +54,19 @@ lx_status check_plan(const lx_plan* p, const lx_bhld* shape) {
   return LX_OK;
 }
 
+// Persistent 128-thread grid of the V quantiser: four CTAs per SM, each over a
+// contiguous range of `per` units.
+bool persistent_grid(long long units, long long* ctas, long long* per) {
+  int dev = 0, sms = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+      sms < 1)
+    return false;
+  const long long want = 4LL * sms;
+  *per = (units + want - 1) / want;
+  *ctas = (units + *per - 1) / *per;
+  return true;
+}
+
 inline lx_status launch_status() {
   return cudaGetLastError() == cudaSuccess ? LX_OK : LX_ERR_CUDA;
 }
@@ -131,7 +144,10 @@ lx_status launch_quant_v(const lx_bhld* V, uint8_t* vc, float* vs, uint32_t* ama
   if (cudaMemsetAsync(amax, 0, sizeof(uint32_t) * BH * D, s) != cudaSuccess) return LX_ERR_CUDA;
   lx::v_absmax_kernel<D><<<(unsigned)(BH * nSpan), 128, 0, s>>>(view(V), amax, (int)V->H, (int)V->L, nSpan);
   if (cudaGetLastError() != cudaSuccess) return LX_ERR_CUDA;
-  lx::v_quant_kernel<D><<<(unsigned)(BH * nB), 128, 0, s>>>(view(V), amax, vc, vs, (int)V->H, (int)V->L, (int)nB);
+  long long ctas = 0, per = 0;
+  if (!persistent_grid(BH * nB, &ctas, &per)) return LX_ERR_CUDA;
+  lx::v_quant_kernel<D><<<(unsigned)ctas, 128, 0, s>>>(view(V), amax, vc, vs, (int)V->H, (int)V->L, (int)nB,
+                                                       (long long)(BH * nB), per);
   return launch_status();
 }
 

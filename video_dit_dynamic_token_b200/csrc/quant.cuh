@@ -95,6 +95,12 @@ __global__ void __launch_bounds__(128) quant_qk_kernel(BhldView q, BhldView k, i
   if (threadIdx.x == 0) S[bh * nB + blk] = a > 0.f ? __fdiv_rn(a, 127.0f) : 1.0f;
 }
 
+template <int NCH>
+__device__ __forceinline__ void load_row_half(const __nv_bfloat16* src, bool valid, uint4 (&v)[NCH]) {
+#pragma unroll
+  for (int i = 0; i < NCH; ++i) v[i] = valid ? ld_stream_v4(src + 8 * i) : make_uint4(0, 0, 0, 0);
+}
+
 // ---------------------------------------------------------------------------
 // V, pass 1: per-channel absmax.  One 128-thread CTA per (b*h, 512-token span);
 // lanes cover 16-byte channel chunks; the CTA folds its rows in shared memory
@@ -134,46 +140,75 @@ __global__ void __launch_bounds__(128) v_absmax_kernel(BhldView v, uint32_t* __r
   }
 }
 
-// V, pass 2: codes.  One 128-thread CTA per (b*h, 64-token block); thread t
-// covers row t/2 and half of the channels, like quant_qk_kernel.  The CTA of
-// block 0 also writes the per-channel scales.
-template <int D>
-__global__ void __launch_bounds__(128) v_quant_kernel(BhldView v, const uint32_t* __restrict__ amax,
-                                                     uint8_t* __restrict__ vc, float* __restrict__ vs, int H, int L,
-                                                     int nB) {
-  constexpr int NCH = D / 16;
-  const long long bh = blockIdx.x / nB;
-  const int blk = (int)(blockIdx.x - bh * nB);
+__device__ __forceinline__ const __nv_bfloat16* v_row_src(const BhldView& v, long long bh, int blk, int H, int row,
+                                                         int col0) {
   const long long b = bh / H, h = bh - b * H;
-  const int t0 = blk * kBlock;
-  const int cnt = min(kBlock, L - t0);
+  return v.p + b * v.sB + h * v.sH + (long long)(blk * kBlock + row) * v.sL + col0;
+}
+
+// V, pass 2: codes.  A unit is one (b*h, 64-token block); each persistent
+// 128-thread CTA walks a contiguous range of units, thread t covering row t/2
+// and half of the channels, with the next unit's rows loaded into a second
+// register set while the current one is converted.  The per-channel
+// reciprocal scales are rebuilt in shared memory when b*h changes; the CTA
+// that converts block 0 of a head also writes the head's channel scales.
+template <int D>
+__global__ void __launch_bounds__(128, 4) v_quant_kernel(BhldView v, const uint32_t* __restrict__ amax,
+                                                        uint8_t* __restrict__ vc, float* __restrict__ vs, int H,
+                                                        int L, int nB, long long nunits, long long units_per_cta) {
+  constexpr int NCH = D / 16;
+  const long long u_begin = (long long)blockIdx.x * units_per_cta;
+  const long long u_end = min(u_begin + units_per_cta, nunits);
+  if (u_begin >= u_end) return;
   __shared__ float inv_s[D];
-  for (int ch = threadIdx.x; ch < D; ch += blockDim.x) {
-    const float a = __uint_as_float(amax[bh * D + ch]);
-    inv_s[ch] = a > 0.f ? __fdiv_rn(448.0f, a) : 0.f;
-    if (blk == 0) vs[bh * D + ch] = a > 0.f ? __fdiv_rn(a, 448.0f) : 1.0f;
-  }
-  __syncthreads();
   const int row = threadIdx.x >> 1, col0 = (threadIdx.x & 1) * (D / 2);
-  if (row >= cnt) return;
-  const __nv_bfloat16* src = v.p + b * v.sB + h * v.sH + (long long)(t0 + row) * v.sL + col0;
-  uint8_t* dst = vc + (bh * L + t0 + row) * D + col0;
-#pragma unroll
-  for (int i = 0; i < NCH; i += 2) {
-    uint32_t o[4];
-#pragma unroll
-    for (int hh = 0; hh < 2; ++hh) {
-      const uint4 x = ld_stream_v4(src + 8 * (i + hh));
-      const uint32_t w[4] = {x.x, x.y, x.z, x.w};
-      const float* iv = inv_s + col0 + 8 * (i + hh);
-      uint32_t p[4];
-#pragma unroll
-      for (int e = 0; e < 4; ++e)
-        p[e] = e4m3x2(__fmul_rn(bf16lo(w[e]), iv[2 * e]), __fmul_rn(bf16hi(w[e]), iv[2 * e + 1]));
-      o[2 * hh] = p[0] | (p[1] << 16);
-      o[2 * hh + 1] = p[2] | (p[3] << 16);
+  uint4 x[NCH], xn[NCH];
+  long long bh = u_begin / nB;
+  int blk = (int)(u_begin - bh * nB);
+  load_row_half<NCH>(v_row_src(v, bh, blk, H, row, col0), row < min(kBlock, L - blk * kBlock), x);
+  long long bh_s = -1;  // head whose scales sit in inv_s
+  for (long long u = u_begin; u < u_end; ++u) {
+    const long long bhn = (u + 1) / nB;
+    const int blkn = (int)(u + 1 - bhn * nB);
+    if (u + 1 < u_end)
+      load_row_half<NCH>(v_row_src(v, bhn, blkn, H, row, col0), row < min(kBlock, L - blkn * kBlock), xn);
+    if (bh != bh_s) {
+      __syncthreads();  // every thread is done with the previous head's scales
+      for (int ch = threadIdx.x; ch < D; ch += blockDim.x) {
+        const float a = __uint_as_float(amax[bh * D + ch]);
+        inv_s[ch] = a > 0.f ? __fdiv_rn(448.0f, a) : 0.f;
+      }
+      __syncthreads();
+      bh_s = bh;
     }
-    *reinterpret_cast<uint4*>(dst + 8 * i) = make_uint4(o[0], o[1], o[2], o[3]);
+    if (blk == 0)
+      for (int ch = threadIdx.x; ch < D; ch += blockDim.x) {
+        const float a = __uint_as_float(amax[bh * D + ch]);
+        vs[bh * D + ch] = a > 0.f ? __fdiv_rn(a, 448.0f) : 1.0f;
+      }
+    if (row < min(kBlock, L - blk * kBlock)) {
+      uint8_t* dst = vc + (bh * L + blk * kBlock + row) * D + col0;
+#pragma unroll
+      for (int i = 0; i < NCH; i += 2) {
+        uint32_t o[4];
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+          const uint32_t w[4] = {x[i + hh].x, x[i + hh].y, x[i + hh].z, x[i + hh].w};
+          const float* iv = inv_s + col0 + 8 * (i + hh);
+          uint32_t p[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e)
+            p[e] = e4m3x2(__fmul_rn(bf16lo(w[e]), iv[2 * e]), __fmul_rn(bf16hi(w[e]), iv[2 * e + 1]));
+          o[2 * hh] = p[0] | (p[1] << 16);
+          o[2 * hh + 1] = p[2] | (p[3] << 16);
+        }
+        *reinterpret_cast<uint4*>(dst + 8 * i) = make_uint4(o[0], o[1], o[2], o[3]);
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < NCH; ++i) x[i] = xn[i];
+    bh = bhn;
+    blk = blkn;
   }
 }
 
