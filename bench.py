@@ -33,7 +33,7 @@ METRIC = "block-sparse attn effective TFLOPS (720p grid, 40x128, keep 10%)"
 # kernel build: the ncu capture in profiles/attn_int8fp8_720p_8heads_ncu.md
 # (8 of the 40 heads; traffic grows with the head count, so x5).  Set to None
 # whenever the attention kernel changes until it is captured again.
-ATTN_DRAM_BYTES_PER_LAUNCH = None
+ATTN_DRAM_BYTES_PER_LAUNCH = 5 * (236.903424e6 + 126.946048e6)
 
 
 def reduce_max(x: float, device) -> float:
