@@ -26,7 +26,14 @@ sys.path.insert(0, ROOT)
 
 WORKLOAD = "720p"
 MODE = "int8fp8"
-METRIC = "block-sparse attn effective TFLOPS (720p grid, 40x128, keep 10%)"
+METRIC = "block-sparse attn ms & effective TFLOPS (720p grid, 40\u00d7128, keep 10%)"
+
+
+def metric_for(workload, H, d, keep):
+    """The headline metric's name; other workloads get the same form."""
+    if workload == WORKLOAD and H == 40 and d == 128 and abs(keep - 0.1) < 1e-12:
+        return METRIC
+    return f"block-sparse attn ms & effective TFLOPS ({workload} grid, {H}\u00d7{d}, keep {keep:g})"
 
 
 # DRAM bytes (read + write) of one full-size attention launch of the current
@@ -124,15 +131,20 @@ def run_ours(args, rank, world, local_rank):
 
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
-    w = synth.WORKLOADS[WORKLOAD]
-    B, H, d, L, keep = w.B, args.heads or w.H, w.d, w.L, w.keep
+    w = synth.WORKLOADS[args.workload]
+    B, H, d, L = w.B, args.heads or w.H, w.d, w.L
+    keep = args.keep if args.keep else w.keep
+    mode = args.mode
     nB = math.ceil(L / 64)
     Q, K, V = synth.make_qkv(B, H, d, w.grid, seed=rank, device=dev)
     k, _, _, plan_ws_bytes = lx.lx_plan_size(B, H, L, d, keep)
     plan = lx.empty_plan(B, H, L, d, keep, dev)
     plan_ws = torch.empty(plan_ws_bytes, dtype=torch.uint8, device=dev)
-    mq = plan_ws[: plan_ws_bytes // 2].view(torch.float32).view(B, H, nB, d)
-    mk = plan_ws[plan_ws_bytes // 2:].view(torch.float32).view(B, H, nB, d)
+    # planner workspace: [means of Q | means of K | scores], 256-byte aligned
+    means = (4 * B * H * nB * d + 255) // 256 * 256
+    mq = plan_ws[:means][: 4 * B * H * nB * d].view(torch.float32).view(B, H, nB, d)
+    mk = plan_ws[means:2 * means][: 4 * B * H * nB * d].view(torch.float32).view(B, H, nB, d)
+    score_ws = plan_ws[2 * means:]
     qc = torch.empty((B, H, L, d), dtype=torch.int8, device=dev)
     kc = torch.empty_like(qc)
     vc = torch.empty((B, H, L, d), dtype=torch.uint8, device=dev)
@@ -143,28 +155,33 @@ def run_ours(args, rank, world, local_rank):
     O = torch.empty_like(Q)
     stream = torch.cuda.current_stream(dev)
     flops = lx.effective_flops(B, H, L, d, keep)
-    launches_per_step = 6  # pool, score+top-k, quant Q/K, V absmax, V quant, attention
-
-    names = ["pool", "score_topk", "quant_qk", "quant_v", "attn"]
+    if mode == "int8fp8":
+        launches_per_step = 6  # pool, score+top-k, quant Q/K, V absmax, V quant, attention
+        names = ["pool", "score_topk", "quant_qk", "quant_v", "attn"]
+    else:
+        launches_per_step = 3  # pool, score+top-k, attention
+        names = ["pool", "score_topk", "attn"]
 
     def step(ev=None):
-        if ev is not None:
-            ev[0].record(stream)
+        marks = iter(range(len(names) + 1))
+        def mark():
+            i = next(marks)
+            if ev is not None:
+                ev[i].record(stream)
+        mark()
         lx.lx_pool_means(Q, K, out=(mq, mk))
-        if ev is not None:
-            ev[1].record(stream)
-        lx.lx_score_topk(mq, mk, L, keep, plan=plan)
-        if ev is not None:
-            ev[2].record(stream)
-        lx.lx_quantize_qk(Q, K, out=(qc, qs, kc, ks))
-        if ev is not None:
-            ev[3].record(stream)
-        lx.lx_quantize_v(V, out=(vc, vs), amax_ws=amax)
-        if ev is not None:
-            ev[4].record(stream)
-        lx.lx_attn_int8fp8(qc, qs, kc, ks, vc, vs, plan, out=O)
-        if ev is not None:
-            ev[5].record(stream)
+        mark()
+        lx.lx_score_topk(mq, mk, L, keep, plan=plan, ws=score_ws)
+        mark()
+        if mode == "int8fp8":
+            lx.lx_quantize_qk(Q, K, out=(qc, qs, kc, ks))
+            mark()
+            lx.lx_quantize_v(V, out=(vc, vs), amax_ws=amax)
+            mark()
+            lx.lx_attn_int8fp8(qc, qs, kc, ks, vc, vs, plan, out=O)
+        else:
+            lx.lx_attn_bf16(Q, K, V, plan, out=O)
+        mark()
 
     for _ in range(args.warmup):
         step()
@@ -173,7 +190,7 @@ def run_ours(args, rank, world, local_rank):
     if st != 0:
         raise RuntimeError(f"device status {st} after warm-up")
 
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(args.steps)]
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(len(names) + 1)] for _ in range(args.steps)]
     sampler = ClockSampler(local_rank) if rank == 0 else None
     if world > 1:
         dist.barrier()
@@ -207,7 +224,7 @@ def run_ours(args, rank, world, local_rank):
         hQ, hK, hV = (x.cpu().pin_memory() for x in (Q, K, V))
         hO = torch.empty(O.shape, dtype=O.dtype).pin_memory()
         # the public host-to-host path: head chunks with copies and kernels overlapped
-        pipe = HostPipeline(B, H, L, d, keep, MODE, heads_per_chunk=args.e2e_heads_per_chunk, device=dev)
+        pipe = HostPipeline(B, H, L, d, keep, mode, heads_per_chunk=args.e2e_heads_per_chunk, device=dev)
 
         def e2e_step():
             pipe.run(hQ, hK, hV, hO, stream=stream)
@@ -233,27 +250,33 @@ def run_ours(args, rank, world, local_rank):
     peaks = _peaks()
     attn_ms = per["attn"]
     achieved = flops / (attn_ms * 1e-3) / 1e12
-    peak = 2.0 * peaks["bf16_sustained"]
+    # dense 8-bit peak = 2 x bf16 (the nominal ratio); bf16 mode against bf16 itself
+    peak = (2.0 if mode == "int8fp8" else 1.0) * peaks["bf16_sustained"]
     plan_bytes = 2 * B * H * L * d * 2 + B * H * nB * k * 4 + B * H * nB * ((nB + 31) // 32) * 4
     plan_ms = per["pool"] + per["score_topk"]
-    # Q/K/V codes read once, O written once (bf16), kept ids
-    attn_bytes = 3 * B * H * L * d + B * H * L * d * 2 + B * H * nB * k * 4
+    # Q/K/V (codes or bf16) read once, O written once (bf16), kept ids
+    esz = 1 if mode == "int8fp8" else 2
+    attn_bytes = 3 * B * H * L * d * esz + B * H * L * d * 2 + B * H * nB * k * 4
     out = {
-        "metric": METRIC, "value": round(value, 2), "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "metric": metric_for(args.workload, H, d, keep), "value": round(value, 2), "unit": "TFLOP/s",
+        "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(ms_step, 4), "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "int8fp8", "data": "synthetic (smooth coarsened N(0,1) field + noise, seeded)",
-        "config": {"workload": f"720p-shaped B={B} H={H} d={d} L={L} keep={keep} mode={MODE}", "k": k, "nB": nB,
+        "vs_baseline": None, "dtype": mode, "data": "synthetic (smooth coarsened N(0,1) field + noise, seeded)",
+        "config": {"workload": f"{args.workload}-shaped B={B} H={H} d={d} L={L} keep={keep} mode={mode}", "k": k,
+                   "nB": nB,
                    "effective_tflop_per_step": round(flops / 1e12, 3), "parallelism": f"replicas x{world}",
                    "l2": "inputs larger than L2 (2.3 GB of Q/K/V per step)"},
         "breakdown_ms": {n: round(v, 4) for n, v in per.items()},
         "attn_ms": round(attn_ms, 4), "attn_effective_tflops": round(achieved, 1),
         "planner_ms": round(plan_ms, 4), "planner_gbs": round(plan_bytes / (plan_ms * 1e-3) / 1e9, 1),
         "planner_hbm_frac": round(plan_bytes / (plan_ms * 1e-3) / 1e9 / peaks["hbm_gbs"], 3),
-        "roofline": {"bound": "tensor", "kernel": "sparse_attn_kernel<128,int8fp8>", "achieved": round(achieved, 1),
+        "roofline": {"bound": "tensor", "kernel": f"sparse_attn_kernel<{d},{mode}>", "achieved": round(achieved, 1),
                      "peak": round(peak, 1), "unit": "TFLOP/s", "frac": round(achieved / peak, 3),
-                     "peak_note": f"2 x {peaks['source']} sustained bf16 ({peaks['bf16_sustained']}) = dense "
-                                  "int8/fp8 by the nominal 2:1 ratio",
-                     "traffic": (None if ATTN_DRAM_BYTES_PER_LAUNCH is None or args.heads
+                     "peak_note": (f"2 x {peaks['source']} sustained bf16 ({peaks['bf16_sustained']}) = dense "
+                                   "int8/fp8 by the nominal 2:1 ratio" if mode == "int8fp8" else
+                                   f"{peaks['source']} sustained bf16 ({peaks['bf16_sustained']})"),
+                     "traffic": (None if ATTN_DRAM_BYTES_PER_LAUNCH is None or args.heads or mode != MODE
+                                 or args.workload != WORKLOAD or args.keep
                                  else int(ATTN_DRAM_BYTES_PER_LAUNCH)),
                      "traffic_note": "ncu dram__bytes_read+write per launch (8-head capture x5)",
                      "algorithmic_bytes": int(attn_bytes)},
@@ -337,6 +360,10 @@ def main():
     ap.add_argument("--e2e-heads-per-chunk", type=int, default=2)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--heads", type=int, default=0, help="fewer heads: a smaller case for profiling only")
+    ap.add_argument("--workload", default=WORKLOAD, choices=["480p", "720p", "long"],
+                    help="grid shape (the headline is 720p; the others are characterisation runs)")
+    ap.add_argument("--mode", default=MODE, choices=["int8fp8", "bf16"])
+    ap.add_argument("--keep", type=float, default=0.0, help="override the workload's keep ratio (sweeps)")
     args = ap.parse_args()
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -355,7 +382,8 @@ def main():
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=__import__("torch").device("cuda", local_rank))
     cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline and not args.heads:
+    if (rank == 0 and world == 1 and not args.no_cpu_baseline and not args.heads and args.workload == WORKLOAD
+            and args.mode == MODE and not args.keep):
         cpu = cpu_oracle_sample()
     out = run_ours(args, rank, world, local_rank)
     if world > 1:

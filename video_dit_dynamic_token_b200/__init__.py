@@ -96,14 +96,21 @@ def lx_pool_means(Q, K, out=None, stream=None):
     return out
 
 
-def lx_score_topk(mq, mk, L, keep, plan: Plan | None = None, stream=None) -> Plan:
+def score_ws_bytes(B, H, nB) -> int:
+    """Scratch of lx_score_topk: the fp32 [B,H,nB,nB] score matrix, 256-byte rounded."""
+    return (4 * B * H * nB * nB + 255) // 256 * 256
+
+
+def lx_score_topk(mq, mk, L, keep, plan: Plan | None = None, ws=None, stream=None) -> Plan:
     lib = _abi.load()
     B, H, nB, D = mq.shape
     if plan is None:
         plan = empty_plan(B, H, L, D, keep, mq.device)
+    if ws is None:
+        ws = torch.empty(score_ws_bytes(B, H, nB), dtype=torch.uint8, device=mq.device)
     cp = plan.c()
-    _check(lib.lx_score_topk(_ptr(mq), _ptr(mk), B, H, L, D, float(keep), ctypes.byref(cp), _stream(stream)),
-           "lx_score_topk")
+    _check(lib.lx_score_topk(_ptr(mq), _ptr(mk), B, H, L, D, float(keep), ctypes.byref(cp), _ptr(ws), ws.numel(),
+                             _stream(stream)), "lx_score_topk")
     return plan
 
 

@@ -38,7 +38,7 @@ _P = ctypes.POINTER
 SIGNATURES = {
     "lx_plan_size": [_c_i64, _c_i64, _c_i64, _c_i64, _dbl, _P(_c_i64), _P(_c_sz), _P(_c_sz), _P(_c_sz)],
     "lx_pool_means": [_P(LxBhld), _P(LxBhld), _vp, _vp, _vp],
-    "lx_score_topk": [_vp, _vp, _c_i64, _c_i64, _c_i64, _c_i64, _dbl, _P(LxPlan), _vp],
+    "lx_score_topk": [_vp, _vp, _c_i64, _c_i64, _c_i64, _c_i64, _dbl, _P(LxPlan), _vp, _c_sz, _vp],
     "lx_sparse_attn_plan": [_P(LxBhld), _P(LxBhld), _dbl, _P(LxPlan), _vp, _c_sz, _vp],
     "lx_quantize_qk": [_P(LxBhld), _P(LxBhld), _vp, _vp, _vp, _vp, _vp],
     "lx_quantize_v": [_P(LxBhld), _vp, _vp, _vp, _vp],

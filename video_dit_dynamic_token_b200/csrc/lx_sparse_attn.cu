@@ -67,6 +67,9 @@ bool persistent_grid(long long units, long long* ctas, long long* per) {
   return true;
 }
 
+// Score workspace of lx_score_topk: fp32 [B*H, nB, nB].
+inline size_t score_ws_bytes(int64_t BH, int64_t nB) { return align256(sizeof(float) * (size_t)(BH * nB * nB)); }
+
 inline lx_status launch_status() {
   return cudaGetLastError() == cudaSuccess ? LX_OK : LX_ERR_CUDA;
 }
@@ -114,17 +117,32 @@ lx_status launch_pool(const lx_bhld* Q, const lx_bhld* K, float* mq, float* mk, 
 }
 
 template <int D>
-lx_status launch_score(const float* mq, const float* mk, int64_t BH, int64_t nB, int64_t k, lx_plan* plan,
-                       cudaStream_t s) {
+lx_status launch_score(const float* mq, const float* mk, int64_t BH, int64_t nB, int64_t k, float* scores,
+                       lx_plan* plan, cudaStream_t s) {
+  // scores: tf32 x3 tensor-core GEMM, one 128 x 256 tile per CTA
+  CUtensorMap tq, tk;
+  const auto f32 = CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
+  if (!make_map(&tq, mq, f32, 4, 1, BH, nB, D, BH * nB * D, nB * D, D, lx::kSgK, lx::kSgM) ||
+      !make_map(&tk, mk, f32, 4, 1, BH, nB, D, BH * nB * D, nB * D, D, lx::kSgK, lx::kSgN))
+    return LX_ERR_CUDA;
+  const size_t gsmem = 1024 + lx::kSgSmem;
+  if (cudaFuncSetAttribute(lx::score_gemm_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)gsmem) !=
+      cudaSuccess)
+    return LX_ERR_CUDA;
+  dim3 ggrid((unsigned)((nB + lx::kSgM - 1) / lx::kSgM), (unsigned)((nB + lx::kSgN - 1) / lx::kSgN), (unsigned)BH);
+  lx::score_gemm_kernel<D><<<ggrid, 128, gsmem, s>>>(tq, tk, scores, (int)nB, kWaitLimitNs);
+  if (cudaGetLastError() != cudaSuccess) return LX_ERR_CUDA;
+  // selection: 8 rows per CTA, one warp per row
   const int ldS = (int)((nB + 31) / 32 * 32);
-  const size_t smem = sizeof(float) * ((size_t)lx::kKeyStages * lx::kKeyChunk * D + (size_t)lx::kScoreRows * ldS +
+  const size_t smem = sizeof(float) * ((size_t)lx::kScoreRows * ldS +
                                        lx::kScoreWarps * (256 + 2 * lx::kCandCap + ldS / 32));
   if (smem > 227 * 1024) return LX_ERR_UNSUPPORTED;
-  if (cudaFuncSetAttribute(lx::score_topk_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+  if (cudaFuncSetAttribute(lx::select_topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
       cudaSuccess)
     return LX_ERR_CUDA;
   dim3 grid((unsigned)((nB + lx::kScoreRows - 1) / lx::kScoreRows), (unsigned)BH);
-  lx::score_topk_kernel<D><<<grid, 32 * lx::kScoreWarps, smem, s>>>(mq, mk, (int)nB, (int)k, plan->idx, plan->mask, ldS, kWaitLimitNs);
+  lx::select_topk_kernel<<<grid, 32 * lx::kScoreWarps, smem, s>>>(scores, (int)nB, (int)k, plan->idx, plan->mask,
+                                                                   ldS);
   return launch_status();
 }
 
@@ -253,7 +271,7 @@ lx_status lx_plan_size(int64_t B, int64_t H, int64_t L, int64_t D, double keep, 
   if (k) *k = kk;
   if (idx_bytes) *idx_bytes = sizeof(int32_t) * (size_t)(B * H * nB * kk);
   if (mask_bytes) *mask_bytes = sizeof(uint32_t) * (size_t)(B * H * nB * ((nB + 31) / 32));
-  if (ws_bytes) *ws_bytes = 2 * align256(sizeof(float) * (size_t)(B * H * nB * D));
+  if (ws_bytes) *ws_bytes = 2 * align256(sizeof(float) * (size_t)(B * H * nB * D)) + score_ws_bytes(B * H, nB);
   return LX_OK;
 }
 
@@ -266,7 +284,7 @@ lx_status lx_pool_means(const lx_bhld* Q, const lx_bhld* K, float* mq, float* mk
 }
 
 lx_status lx_score_topk(const float* mq, const float* mk, int64_t B, int64_t H, int64_t L, int64_t D, double keep,
-                        lx_plan* plan, cudaStream_t stream) {
+                        lx_plan* plan, void* ws, size_t ws_bytes, cudaStream_t stream) {
   int64_t k = 0;
   lx_status st = lx_plan_size(B, H, L, D, keep, &k, nullptr, nullptr, nullptr);
   if (st != LX_OK) return st;
@@ -274,14 +292,17 @@ lx_status lx_score_topk(const float* mq, const float* mk, int64_t B, int64_t H, 
   if (!al16(mq) || !al16(mk) || !al16(plan->idx) || (plan->mask && !al16(plan->mask))) return LX_ERR_ALIGN;
   const int64_t nB = n_blocks(L);
   if (nB > kMaxPlannerNB) return LX_ERR_UNSUPPORTED;
+  if (!ws || ws_bytes < score_ws_bytes(B * H, nB)) return LX_ERR_WORKSPACE;
+  if (!al16(ws)) return LX_ERR_ALIGN;
   plan->B = B;
   plan->H = H;
   plan->L = L;
   plan->nB = nB;
   plan->k = k;
   plan->block = LX_BLOCK;
-  return D == 128 ? launch_score<128>(mq, mk, B * H, nB, k, plan, stream)
-                  : launch_score<64>(mq, mk, B * H, nB, k, plan, stream);
+  float* scores = reinterpret_cast<float*>(ws);
+  return D == 128 ? launch_score<128>(mq, mk, B * H, nB, k, scores, plan, stream)
+                  : launch_score<64>(mq, mk, B * H, nB, k, scores, plan, stream);
 }
 
 lx_status lx_sparse_attn_plan(const lx_bhld* Q, const lx_bhld* K, double keep, lx_plan* plan, void* ws,
@@ -294,10 +315,13 @@ lx_status lx_sparse_attn_plan(const lx_bhld* Q, const lx_bhld* K, double keep, l
   if (!ws || ws_bytes < need) return LX_ERR_WORKSPACE;
   if (!al16(ws)) return LX_ERR_ALIGN;
   if (n_blocks(Q->L) > kMaxPlannerNB) return LX_ERR_UNSUPPORTED;
+  // workspace: [block means of Q | block means of K | scores], 256-byte aligned
+  const size_t means = align256(sizeof(float) * (size_t)(Q->B * Q->H * n_blocks(Q->L) * Q->D));
   float* mq = reinterpret_cast<float*>(ws);
-  float* mk = reinterpret_cast<float*>(reinterpret_cast<char*>(ws) + need / 2);
+  float* mk = reinterpret_cast<float*>(reinterpret_cast<char*>(ws) + means);
+  char* sc = reinterpret_cast<char*>(ws) + 2 * means;
   if ((st = lx_pool_means(Q, K, mq, mk, stream)) != LX_OK) return st;
-  return lx_score_topk(mq, mk, Q->B, Q->H, Q->L, Q->D, keep, plan, stream);
+  return lx_score_topk(mq, mk, Q->B, Q->H, Q->L, Q->D, keep, plan, sc, need - 2 * means, stream);
 }
 
 lx_status lx_quantize_qk(const lx_bhld* Q, const lx_bhld* K, int8_t* qc, float* qs, int8_t* kc, float* ks,

@@ -1,5 +1,5 @@
-// Planner kernels: block-mean pooling of Q and K (step a1) and pooled-mean
-// scoring with per-row top-k selection (step a2).
+// Planner kernels: block-mean pooling of Q and K (step a1); pooled-mean
+// scores on the tensor cores and per-row top-k selection (step a2).
 //
 // "600倍加速，720p视频实时生成！单卡也能带的动14B模型", §动态稀疏量化注意力: the
 // importance of each attention tile is estimated from block-level means of Q
@@ -87,132 +87,167 @@ __global__ void __launch_bounds__(256) pool_means_kernel(BhldView q, BhldView k,
 }
 
 // ---------------------------------------------------------------------------
-// a2: one CTA per (b*h, 16 query-block rows), 16 warps.
-//  Scoring: every warp computes all 16 rows for its share of the key blocks
-//  (two keys at a time, so eight independent FMA chains per lane).
-//  Lane = (row group rg in 0..3) x (d-slice ds in 0..7); a lane keeps the 4
-//  rows x D/8 pooled-query values of its slice in registers and reads the
-//  pooled key in 16-byte pieces (slices are interleaved so the 8 slices of one
-//  key are one contiguous 128-byte wavefront); partial dots are folded across
-//  the 8 slices with 4 shuffles.  Scores land in shared memory (fp32).
-//  Selection: one warp per row.  Scores are bucketed into 256 monotone
-//  buckets between the row min and max; the bucket holding the k-th largest is
-//  resolved exactly by ranking its members with the (score desc, index asc)
-//  order; the kept ids are emitted in ascending order with a ballot scan that
-//  also yields the bitmask words.
-constexpr int kScoreRows = 16;
-constexpr int kKeyChunk = 32;
+// a2, scores: S[b,h,i,j] = Mq[b,h,i,:] . Mk[b,h,j,:] for all block pairs of a
+// head, on the tensor cores with fp32-level accuracy.  One 128-thread CTA
+// computes a 128-row x 128-key tile.  Each 32-dimension chunk of the pooled
+// means arrives by TMA (fp32, 128-byte swizzle) into one of two chunk buffers
+// (the next chunk loads while the current one is used) and is split in place
+// into a tf32-exact high part h = x rounded to 10 mantissa bits, plus the
+// remainder l = x - h (exact in fp32) in a third buffer; three kind::tf32 MMAs (h.h + h.l + l.h) then
+// accumulate in TMEM, leaving only the l.l term and the tf32 truncation of l,
+// about 2^-22 of each product.  The tile leaves through shared memory, one
+// 128-byte row segment per warp store.  Dividing by sqrt(d) changes no
+// ranking and is left out.
+constexpr int kSgM = 128, kSgN = 128, kSgK = 32;  // rows, keys, dimensions per chunk
+constexpr int kSgA = kSgM * kSgK * 4;             // bytes of one A chunk (16 KB)
+constexpr int kSgB = kSgN * kSgK * 4;             // bytes of one B chunk (16 KB)
+constexpr int kSgRaw = kSgA + kSgB;               // one raw chunk (A then B)
+constexpr int kSgSmem = 3 * kSgRaw;              // two chunk buffers (raw, then high part) + low parts
+constexpr uint32_t kSgIdesc = instr_desc(IDESC_DF32, IDESC_TF32, IDESC_TF32, 0, 0, kSgM, kSgN);
+
+__device__ __forceinline__ float tf32_high(float v) {
+  return __uint_as_float((__float_as_uint(v) + 0x1000u) & 0xFFFFE000u);
+}
+
+template <int D>
+__global__ void __launch_bounds__(128, 2) score_gemm_kernel(const __grid_constant__ CUtensorMap tmQ,
+                                                           const __grid_constant__ CUtensorMap tmK,
+                                                           float* __restrict__ S, int nB,
+                                                           unsigned long long limit_ns) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* raw = sm;                     // 2 x [A chunk | B chunk]: TMA destinations, then high parts
+  uint8_t* lo = sm + 2 * kSgRaw;         // [A | B] low parts, same swizzled layout
+  __shared__ uint64_t bar_ld[2], bar_mma;
+  __shared__ uint32_t tmem_slot;
+  __shared__ int never_abort;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int m0 = blockIdx.x * kSgM, n0 = blockIdx.y * kSgN, bh = blockIdx.z;
+  constexpr int NK = D / kSgK;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar_ld[0], 1);
+    mbar_init(&bar_ld[1], 1);
+    mbar_init(&bar_mma, 1);
+    never_abort = 0;
+    fence_barrier_init();
+  }
+  if (warp == 0) {
+    tmem_alloc(&tmem_slot, kSgN);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tbase = tmem_slot;
+  // every exit from the chunk loop is CTA-uniform (__syncthreads_and), so no
+  // thread is left at a barrier; loads and MMAs in flight are drained below
+  int issued_ld = 0, issued_mma = 0;  // chunks whose TMA loads / MMAs thread 0 issued
+  if (threadIdx.x == 0) {
+    mbar_arrive_expect_tx(&bar_ld[0], kSgRaw);
+    tma_load_4d(raw, &tmQ, &bar_ld[0], 0, m0, bh, 0);
+    tma_load_4d(raw + kSgA, &tmK, &bar_ld[0], 0, n0, bh, 0);
+    issued_ld = 1;
+  }
+  bool ok = true;
+  for (int kc = 0; kc < NK; ++kc) {
+    const int rb = kc & 1;
+    uint8_t* hi = raw + rb * kSgRaw;
+    // chunk kc has landed, and the previous chunk's MMAs are done with the low
+    // buffer and with the other chunk buffer, which chunk kc+1 now loads into
+    bool w = mbar_wait(&bar_ld[rb], (kc >> 1) & 1, &never_abort, limit_ns);
+    w = w && (kc == 0 || mbar_wait(&bar_mma, (kc - 1) & 1, &never_abort, limit_ns));
+    ok = __syncthreads_and(ok && w) != 0;
+    if (!ok) break;
+    if (threadIdx.x == 0 && kc + 1 < NK) {
+      uint8_t* nxt = raw + (rb ^ 1) * kSgRaw;
+      mbar_arrive_expect_tx(&bar_ld[rb ^ 1], kSgRaw);
+      tma_load_4d(nxt, &tmQ, &bar_ld[rb ^ 1], (kc + 1) * kSgK, m0, bh, 0);
+      tma_load_4d(nxt + kSgA, &tmK, &bar_ld[rb ^ 1], (kc + 1) * kSgK, n0, bh, 0);
+      issued_ld = kc + 2;
+    }
+    float4* h4 = reinterpret_cast<float4*>(hi);
+    float4* l4 = reinterpret_cast<float4*>(lo);
+    for (int i = threadIdx.x; i < kSgRaw / 16; i += blockDim.x) {
+      const float4 x = h4[i];
+      const float4 h = make_float4(tf32_high(x.x), tf32_high(x.y), tf32_high(x.z), tf32_high(x.w));
+      h4[i] = h;
+      l4[i] = make_float4(x.x - h.x, x.y - h.y, x.z - h.z, x.w - h.w);
+    }
+    fence_proxy_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      tc_fence_after();
+#pragma unroll
+      for (int ks = 0; ks < kSgK / 8; ++ks) {  // 8 tf32 values = 32 bytes per MMA
+        const uint64_t ah = smem_desc(smem_u32(hi) + ks * 32, 16, 8 * 128, SW_128B);
+        const uint64_t al = smem_desc(smem_u32(lo) + ks * 32, 16, 8 * 128, SW_128B);
+        const uint64_t bhd = smem_desc(smem_u32(hi + kSgA) + ks * 32, 16, 8 * 128, SW_128B);
+        const uint64_t bld = smem_desc(smem_u32(lo + kSgA) + ks * 32, 16, 8 * 128, SW_128B);
+        mma_ss<KIND_TF32>(tbase, ah, bhd, kSgIdesc, (kc > 0 || ks > 0) ? 1u : 0u);
+        mma_ss<KIND_TF32>(tbase, ah, bld, kSgIdesc, 1u);
+        mma_ss<KIND_TF32>(tbase, al, bhd, kSgIdesc, 1u);
+      }
+      mma_commit(&bar_mma);
+      issued_mma = kc + 1;
+    }
+  }
+  if (ok) ok = __syncthreads_and(mbar_wait(&bar_mma, (NK - 1) & 1, &never_abort, limit_ns)) != 0;
+  if (!ok) {
+    if (threadIdx.x == 0) {
+      report_error(-6);
+      // drain what is still in flight before the CTA exits and frees TMEM
+      for (int c = issued_ld - 2 < 0 ? 0 : issued_ld - 2; c < issued_ld; ++c)
+        mbar_wait(&bar_ld[c & 1], (c >> 1) & 1, &never_abort, limit_ns);
+      if (issued_mma > 0) mbar_wait(&bar_mma, (issued_mma - 1) & 1, &never_abort, limit_ns);
+    }
+  } else {
+    tc_fence_after();
+    // warp w holds tile rows 32w .. 32w+31 (TMEM lanes of its quarter); each
+    // 32 x 32 block goes through a padded shared tile and out row by row, one
+    // 128-byte segment per store
+    float* tile = reinterpret_cast<float*>(lo) + warp * 32 * 33;
+#pragma unroll 1
+    for (int cc = 0; cc < kSgN; cc += 32) {
+      uint32_t v[32];
+      tmem_ld32(tbase + ((uint32_t)(warp * 32) << 16) + cc, v);
+      tmem_wait_ld();
+#pragma unroll
+      for (int i = 0; i < 32; ++i) tile[lane * 33 + i] = __uint_as_float(v[i]);
+      __syncwarp();
+      const int j = n0 + cc + lane;
+#pragma unroll 4
+      for (int r = 0; r < 32; ++r) {
+        const int row = m0 + warp * 32 + r;
+        if (row < nB && j < nB) S[((long long)bh * nB + row) * nB + j] = tile[r * 33 + lane];
+      }
+      __syncwarp();
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tbase, kSgN);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// a2, selection: one 256-thread CTA per (b*h, 8 query-block rows); the 8
+// score rows are copied from the score workspace into shared memory and each
+// warp selects one row: scores are bucketed into 256 monotone buckets between
+// the row min and max; the bucket holding the k-th largest is resolved
+// exactly by ranking its members with the (score desc, index asc) order; the
+// kept ids are emitted in ascending order with a ballot scan that also yields
+// the bitmask words.
+constexpr int kScoreRows = 8;
 constexpr int kCandCap = 64;
+constexpr int kScoreWarps = 8;
 
 __device__ __forceinline__ uint32_t lanemask_lt() {
   uint32_t m;
   asm("mov.u32 %0, %%lanemask_lt;" : "=r"(m));
   return m;
-}
-
-// Pooled keys stream through a ring of shared-memory stages filled by bulk
-// copies (one thread issues, every warp reads), so the L2 latency of one chunk
-// hides behind the arithmetic on the previous ones.
-constexpr int kKeyStages = 3;
-constexpr int kScoreWarps = 16;  // 512 threads share one CTA's score rows
-
-template <int D>
-__device__ __forceinline__ void score_rows(const float* __restrict__ Mq, const float* __restrict__ Mk, int nB,
-                                           int row0, int nrows, float* sS, int ldS, float* sK, uint64_t* kfull,
-                                           uint64_t* kempty, const volatile int* abort_flag,
-                                           unsigned long long limit_ns) {
-  constexpr int DS = D / 8;   // values per lane slice
-  constexpr int NQ = DS / 4;  // float4 pieces per slice
-  constexpr int CHUNK_FLOATS = kKeyChunk * D;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int rg = lane >> 3, ds = lane & 7;
-  const int nchunks = (nB + kKeyChunk - 1) / kKeyChunk;
-  // Slice ds covers d = 32*qq + 4*ds + e  (qq < NQ, e < 4).
-  float qv[4][DS];
-#pragma unroll
-  for (int r = 0; r < 4; ++r) {
-    const int row = row0 + rg * 4 + r;
-#pragma unroll
-    for (int qq = 0; qq < NQ; ++qq) {
-      float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-      if (row - row0 < nrows) v = *reinterpret_cast<const float4*>(Mq + (long long)row * D + 32 * qq + 4 * ds);
-      qv[r][4 * qq] = v.x;
-      qv[r][4 * qq + 1] = v.y;
-      qv[r][4 * qq + 2] = v.z;
-      qv[r][4 * qq + 3] = v.w;
-    }
-  }
-  auto issue = [&](int ch) {
-    const int st = ch % kKeyStages;
-    const int nk = min(kKeyChunk, nB - ch * kKeyChunk);
-    mbar_arrive_expect_tx(&kfull[st], (uint32_t)(nk * D * 4));
-    bulk_load(sK + st * CHUNK_FLOATS, Mk + (long long)ch * kKeyChunk * D, (uint32_t)(nk * D * 4), &kfull[st]);
-  };
-  if (threadIdx.x == 0)
-    for (int ch = 0; ch < min(kKeyStages, nchunks); ++ch) issue(ch);
-  bool ok = true;
-  for (int ch = 0; ch < nchunks; ++ch) {
-    const int st = ch % kKeyStages;
-    const int j0 = ch * kKeyChunk;
-    const int nk = min(kKeyChunk, nB - j0);
-    if (!mbar_wait(&kfull[st], (ch / kKeyStages) & 1, abort_flag, limit_ns)) {
-      ok = false;
-      break;
-    }
-    const float* sKc = sK + st * CHUNK_FLOATS;
-    // warp w handles keys jj = w and w + 16 of the chunk, together
-    {
-      const int ja = warp, jb = warp + kScoreWarps;
-      const bool va = ja < nk, vb = jb < nk;
-      const float* ka = sKc + (va ? ja : 0) * D;
-      const float* kb = sKc + (vb ? jb : 0) * D;
-      float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-#pragma unroll
-      for (int qq = 0; qq < NQ; ++qq) {
-        const float4 xa = *reinterpret_cast<const float4*>(ka + 32 * qq + 4 * ds);
-        const float4 xb = *reinterpret_cast<const float4*>(kb + 32 * qq + 4 * ds);
-#pragma unroll
-        for (int r = 0; r < 4; ++r) {
-          acc[0][r] = fmaf(qv[r][4 * qq], xa.x, acc[0][r]);
-          acc[1][r] = fmaf(qv[r][4 * qq], xb.x, acc[1][r]);
-          acc[0][r] = fmaf(qv[r][4 * qq + 1], xa.y, acc[0][r]);
-          acc[1][r] = fmaf(qv[r][4 * qq + 1], xb.y, acc[1][r]);
-          acc[0][r] = fmaf(qv[r][4 * qq + 2], xa.z, acc[0][r]);
-          acc[1][r] = fmaf(qv[r][4 * qq + 2], xb.z, acc[1][r]);
-          acc[0][r] = fmaf(qv[r][4 * qq + 3], xa.w, acc[0][r]);
-          acc[1][r] = fmaf(qv[r][4 * qq + 3], xb.w, acc[1][r]);
-        }
-      }
-      // fold the 8 slices: after three stages lane ds holds row 2*(ds>>2&1)+(ds>>1&1)
-      const bool hi4 = (ds & 4) != 0, hi2 = (ds & 2) != 0;
-      const int r = 2 * (hi4 ? 1 : 0) + (hi2 ? 1 : 0);
-#pragma unroll
-      for (int kx = 0; kx < 2; ++kx) {
-        float s0 = hi4 ? acc[kx][0] : acc[kx][2], s1 = hi4 ? acc[kx][1] : acc[kx][3];
-        float k0 = hi4 ? acc[kx][2] : acc[kx][0], k1 = hi4 ? acc[kx][3] : acc[kx][1];
-        k0 += __shfl_xor_sync(0xffffffffu, s0, 4);
-        k1 += __shfl_xor_sync(0xffffffffu, s1, 4);
-        float s2 = hi2 ? k0 : k1;
-        float k2 = hi2 ? k1 : k0;
-        k2 += __shfl_xor_sync(0xffffffffu, s2, 2);
-        k2 += __shfl_xor_sync(0xffffffffu, k2, 1);
-        const int jj = kx ? jb : ja;
-        if ((ds & 1) == 0 && (kx ? vb : va)) sS[(rg * 4 + r) * ldS + j0 + jj] = k2;
-      }
-    }
-    __syncwarp();
-    if (lane == 0) mbar_arrive(&kempty[st]);
-    // refill this stage with chunk ch + kKeyStages once all warps are done with it
-    if (threadIdx.x == 0 && ch + kKeyStages < nchunks) {
-      if (!mbar_wait(&kempty[st], (ch / kKeyStages) & 1, abort_flag, limit_ns)) {
-        ok = false;
-        break;
-      }
-      issue(ch + kKeyStages);
-    }
-  }
-  if (!ok) report_error(-6);
-  __syncthreads();
 }
 
 __device__ __forceinline__ int score_bucket(float s, float mn, float scale) {
@@ -353,34 +388,24 @@ __device__ int select_row(const float* __restrict__ s, int nB, int k, int* hist,
   return written;
 }
 
-template <int D>
-__global__ void __launch_bounds__(512, 1) score_topk_kernel(const float* __restrict__ Mq, const float* __restrict__ Mk,
-                                                           int nB, int k, int32_t* __restrict__ idx,
-                                                           uint32_t* __restrict__ mask, int ldS,
-                                                           unsigned long long limit_ns) {
+__global__ void __launch_bounds__(32 * kScoreWarps) select_topk_kernel(const float* __restrict__ S, int nB, int k,
+                                                                      int32_t* __restrict__ idx,
+                                                                      uint32_t* __restrict__ mask, int ldS) {
   extern __shared__ __align__(16) float smem_f[];
-  float* sK = smem_f;                                              // kKeyStages x [32][D]
-  float* sS = sK + kKeyStages * kKeyChunk * D;                     // [16][ldS]
+  float* sS = smem_f;                                                        // [8][ldS]
   int* hist = reinterpret_cast<int*>(sS + kScoreRows * ldS);                 // warps x 256
   float* cand_s = reinterpret_cast<float*>(hist + kScoreWarps * 256);       // warps x 64
   int* cand_j = reinterpret_cast<int*>(cand_s + kScoreWarps * kCandCap);    // warps x 64
   uint32_t* selbits = reinterpret_cast<uint32_t*>(cand_j + kScoreWarps * kCandCap);  // warps x ldS/32
-  __shared__ uint64_t kfull[kKeyStages], kempty[kKeyStages];
-  __shared__ int never_abort;
-  if (threadIdx.x == 0) {
-    for (int i = 0; i < kKeyStages; ++i) {
-      mbar_init(&kfull[i], 1);
-      mbar_init(&kempty[i], kScoreWarps);
-    }
-    never_abort = 0;
-    fence_barrier_init();
-  }
-  __syncthreads();
   const long long bh = blockIdx.y;
   const int row0 = blockIdx.x * kScoreRows;
   const int nrows = min(kScoreRows, nB - row0);
-  score_rows<D>(Mq + bh * nB * D, Mk + bh * nB * D, nB, row0, nrows, sS, ldS, sK, kfull, kempty, &never_abort,
-                limit_ns);
+  const float* src = S + (bh * nB + row0) * (long long)nB;
+  for (int i = threadIdx.x; i < nrows * nB; i += blockDim.x) {
+    const int r = i / nB, j = i - r * nB;
+    sS[r * ldS + j] = src[i];
+  }
+  __syncthreads();
   const int warp = threadIdx.x >> 5;
   const int nW = (nB + 31) >> 5;
   for (int r = warp; r < nrows; r += kScoreWarps) {

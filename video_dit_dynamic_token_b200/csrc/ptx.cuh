@@ -152,7 +152,7 @@ __device__ __forceinline__ void tc_fence_after() {
 }
 
 // ---------------------------------------------------------------- tcgen05: MMA
-enum MmaKind { KIND_F16 = 0, KIND_I8 = 1, KIND_F8F6F4 = 2 };
+enum MmaKind { KIND_F16 = 0, KIND_I8 = 1, KIND_F8F6F4 = 2, KIND_TF32 = 3 };
 
 template <int KIND>
 __device__ __forceinline__ void mma_ss(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
@@ -166,6 +166,12 @@ __device__ __forceinline__ void mma_ss(uint32_t d_tmem, uint64_t adesc, uint64_t
   } else if constexpr (KIND == KIND_I8) {
     asm volatile(
         "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\ttcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, "
+        "p;\n\t}" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+  } else if constexpr (KIND == KIND_TF32) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\ttcgen05.mma.cta_group::1.kind::tf32 [%0], %1, %2, %3, "
         "p;\n\t}" ::"r"(d_tmem),
         "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
         : "memory");
@@ -304,7 +310,7 @@ __host__ __device__ constexpr uint32_t instr_desc(uint32_t dfmt, uint32_t afmt, 
          ((M >> 4) << 24);
 }
 constexpr uint32_t IDESC_DF32 = 1, IDESC_DS32 = 2;
-constexpr uint32_t IDESC_BF16 = 1, IDESC_S8 = 1, IDESC_E4M3 = 0;
+constexpr uint32_t IDESC_BF16 = 1, IDESC_S8 = 1, IDESC_E4M3 = 0, IDESC_TF32 = 2;
 
 // Byte offset of the 16-byte chunk `chunk` of row `row` inside a K-major
 // swizzled atom whose rows are `row_bytes` (128, 64 or 32) long; the XOR
