@@ -81,7 +81,8 @@ typedef struct lx_plan {
 /* Sizes of a plan.  k = clamp(ceil(keep*nB - 1e-6), 1, nB) with nB = ceil(L/64);
  * idx_bytes / mask_bytes size the plan arrays; ws_bytes sizes the workspace of
  * lx_sparse_attn_plan: two fp32 [B,H,nB,D] block-mean arrays followed by the
- * fp32 [B,H,nB,nB] score matrix, each rounded up to 256 bytes.
+ * fp32 [B,H,nB,ldS] score matrix (ldS = nB rounded up to a multiple of 32), each
+ * rounded up to 256 bytes.
  * keep must lie in (0, 1].  Any output pointer may be NULL. */
 lx_status lx_plan_size(int64_t B, int64_t H, int64_t L, int64_t D, double keep, int64_t* k, size_t* idx_bytes,
                        size_t* mask_bytes, size_t* ws_bytes);
@@ -96,8 +97,9 @@ lx_status lx_pool_means(const lx_bhld* Q, const lx_bhld* K, float* mq, float* mk
  * with the largest mean(Q_i).mean(K_j)/sqrt(D), ties to the lower index,
  * ascending.  plan->idx/mask must be set by the caller; the call fills
  * plan->B, H, L, nB, k and block.  nB must not exceed 2176 (L <= 139264).
- * ws: scratch for the fp32 [B,H,nB,nB] score matrix, at least
- * 4*B*H*nB*nB bytes (rounded up to 256), 16-byte aligned (LX_ERR_WORKSPACE /
+ * ws: scratch for the fp32 [B,H,nB,ldS] score matrix (ldS = nB rounded up to a
+ * multiple of 32), at least 4*B*H*nB*ldS bytes (rounded up to 256), 16-byte
+ * aligned (LX_ERR_WORKSPACE /
  * LX_ERR_ALIGN otherwise).  The scores are computed on the tensor cores in
  * three tf32 products (high.high + high.low + low.high of each fp32 mean), which
  * keeps them within about 1e-6 relative of the fp32 dot products. */

@@ -60,7 +60,9 @@ def test_plan_size_matches_oracle_k(lib, L, keep):
     assert k == oracle.keep_count(nB, keep)
     assert ib == 4 * 40 * nB * k
     assert mb == 4 * 40 * nB * ((nB + 31) // 32)
-    assert wb >= 2 * 4 * 40 * nB * 128
+    # two fp32 block-mean arrays, then the fp32 scores with rows padded to 32 floats
+    a256 = lambda n: (n + 255) // 256 * 256
+    assert wb == 2 * a256(4 * 40 * nB * 128) + a256(4 * 40 * nB * ((nB + 31) // 32 * 32))
 
 
 def test_plan_size_rejects(lib):

@@ -97,8 +97,10 @@ def lx_pool_means(Q, K, out=None, stream=None):
 
 
 def score_ws_bytes(B, H, nB) -> int:
-    """Scratch of lx_score_topk: the fp32 [B,H,nB,nB] score matrix, 256-byte rounded."""
-    return (4 * B * H * nB * nB + 255) // 256 * 256
+    """Scratch of lx_score_topk: the fp32 [B,H,nB,ldS] score matrix (ldS = nB
+    rounded up to 32), 256-byte rounded."""
+    ldS = (nB + 31) // 32 * 32
+    return (4 * B * H * nB * ldS + 255) // 256 * 256
 
 
 def lx_score_topk(mq, mk, L, keep, plan: Plan | None = None, ws=None, stream=None) -> Plan:

@@ -67,8 +67,12 @@ bool persistent_grid(long long units, long long* ctas, long long* per) {
   return true;
 }
 
-// Score workspace of lx_score_topk: fp32 [B*H, nB, nB].
-inline size_t score_ws_bytes(int64_t BH, int64_t nB) { return align256(sizeof(float) * (size_t)(BH * nB * nB)); }
+// Score workspace of lx_score_topk: fp32 [B*H, nB, ldS], rows padded to a
+// multiple of 32 floats so that each starts on a 128-byte boundary.
+inline int64_t score_ld(int64_t nB) { return (nB + 31) / 32 * 32; }
+inline size_t score_ws_bytes(int64_t BH, int64_t nB) {
+  return align256(sizeof(float) * (size_t)(BH * nB * score_ld(nB)));
+}
 
 inline lx_status launch_status() {
   return cudaGetLastError() == cudaSuccess ? LX_OK : LX_ERR_CUDA;
@@ -130,10 +134,10 @@ lx_status launch_score(const float* mq, const float* mk, int64_t BH, int64_t nB,
       cudaSuccess)
     return LX_ERR_CUDA;
   dim3 ggrid((unsigned)((nB + lx::kSgM - 1) / lx::kSgM), (unsigned)((nB + lx::kSgN - 1) / lx::kSgN), (unsigned)BH);
-  lx::score_gemm_kernel<D><<<ggrid, 128, gsmem, s>>>(tq, tk, scores, (int)nB, kWaitLimitNs);
+  const int ldS = (int)score_ld(nB);
+  lx::score_gemm_kernel<D><<<ggrid, 128, gsmem, s>>>(tq, tk, scores, (int)nB, ldS, kWaitLimitNs);
   if (cudaGetLastError() != cudaSuccess) return LX_ERR_CUDA;
   // selection: 8 rows per CTA, one warp per row
-  const int ldS = (int)((nB + 31) / 32 * 32);
   const size_t smem = sizeof(float) * ((size_t)lx::kScoreRows * ldS +
                                        lx::kScoreWarps * (256 + 2 * lx::kCandCap + ldS / 32));
   if (smem > 227 * 1024) return LX_ERR_UNSUPPORTED;
@@ -142,7 +146,7 @@ lx_status launch_score(const float* mq, const float* mk, int64_t BH, int64_t nB,
     return LX_ERR_CUDA;
   dim3 grid((unsigned)((nB + lx::kScoreRows - 1) / lx::kScoreRows), (unsigned)BH);
   lx::select_topk_kernel<<<grid, 32 * lx::kScoreWarps, smem, s>>>(scores, (int)nB, (int)k, plan->idx, plan->mask,
-                                                                   ldS);
+                                                                   ldS, kWaitLimitNs);
   return launch_status();
 }
 

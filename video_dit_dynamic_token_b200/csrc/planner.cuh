@@ -96,8 +96,9 @@ __global__ void __launch_bounds__(256) pool_means_kernel(BhldView q, BhldView k,
 // remainder l = x - h (exact in fp32) in a third buffer; three kind::tf32 MMAs (h.h + h.l + l.h) then
 // accumulate in TMEM, leaving only the l.l term and the tf32 truncation of l,
 // about 2^-22 of each product.  The tile leaves through shared memory, one
-// 128-byte row segment per warp store.  Dividing by sqrt(d) changes no
-// ranking and is left out.
+// 128-byte row segment per warp store; rows are ldS = nB rounded up to 32
+// floats apart, so that each starts on a 128-byte boundary (columns nB..ldS-1
+// are never written).  Dividing by sqrt(d) changes no ranking and is left out.
 constexpr int kSgM = 128, kSgN = 128, kSgK = 32;  // rows, keys, dimensions per chunk
 constexpr int kSgA = kSgM * kSgK * 4;             // bytes of one A chunk (16 KB)
 constexpr int kSgB = kSgN * kSgK * 4;             // bytes of one B chunk (16 KB)
@@ -112,7 +113,7 @@ __device__ __forceinline__ float tf32_high(float v) {
 template <int D>
 __global__ void __launch_bounds__(128, 2) score_gemm_kernel(const __grid_constant__ CUtensorMap tmQ,
                                                            const __grid_constant__ CUtensorMap tmK,
-                                                           float* __restrict__ S, int nB,
+                                                           float* __restrict__ S, int nB, int ldS,
                                                            unsigned long long limit_ns) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -219,7 +220,7 @@ __global__ void __launch_bounds__(128, 2) score_gemm_kernel(const __grid_constan
 #pragma unroll 4
       for (int r = 0; r < 32; ++r) {
         const int row = m0 + warp * 32 + r;
-        if (row < nB && j < nB) S[((long long)bh * nB + row) * nB + j] = tile[r * 33 + lane];
+        if (row < nB && j < nB) S[((long long)bh * nB + row) * ldS + j] = tile[r * 33 + lane];
       }
       __syncwarp();
     }
@@ -234,8 +235,8 @@ __global__ void __launch_bounds__(128, 2) score_gemm_kernel(const __grid_constan
 
 // ---------------------------------------------------------------------------
 // a2, selection: one 256-thread CTA per (b*h, 8 query-block rows); the 8
-// score rows are copied from the score workspace into shared memory and each
-// warp selects one row: scores are bucketed into 256 monotone buckets between
+// score rows (contiguous in the workspace, ldS floats apart) arrive in shared
+// memory by one bulk copy, and each warp selects one row: scores are bucketed into 256 monotone buckets between
 // the row min and max; the bucket holding the k-th largest is resolved
 // exactly by ranking its members with the (score desc, index asc) order; the
 // kept ids are emitted in ascending order with a ballot scan that also yields
@@ -390,22 +391,39 @@ __device__ int select_row(const float* __restrict__ s, int nB, int k, int* hist,
 
 __global__ void __launch_bounds__(32 * kScoreWarps) select_topk_kernel(const float* __restrict__ S, int nB, int k,
                                                                       int32_t* __restrict__ idx,
-                                                                      uint32_t* __restrict__ mask, int ldS) {
+                                                                      uint32_t* __restrict__ mask, int ldS,
+                                                                      unsigned long long limit_ns) {
   extern __shared__ __align__(16) float smem_f[];
   float* sS = smem_f;                                                        // [8][ldS]
   int* hist = reinterpret_cast<int*>(sS + kScoreRows * ldS);                 // warps x 256
   float* cand_s = reinterpret_cast<float*>(hist + kScoreWarps * 256);       // warps x 64
   int* cand_j = reinterpret_cast<int*>(cand_s + kScoreWarps * kCandCap);    // warps x 64
   uint32_t* selbits = reinterpret_cast<uint32_t*>(cand_j + kScoreWarps * kCandCap);  // warps x ldS/32
+  __shared__ uint64_t bar_ld;
+  __shared__ int never_abort;
   const long long bh = blockIdx.y;
   const int row0 = blockIdx.x * kScoreRows;
   const int nrows = min(kScoreRows, nB - row0);
-  const float* src = S + (bh * nB + row0) * (long long)nB;
-  for (int i = threadIdx.x; i < nrows * nB; i += blockDim.x) {
-    const int r = i / nB, j = i - r * nB;
-    sS[r * ldS + j] = src[i];
+  // nrows * ldS * 4 bytes: a multiple of 128, from a 128-byte aligned row
+  const uint32_t bytes = (uint32_t)(nrows * ldS) * 4u;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar_ld, 1);
+    never_abort = 0;
+    fence_barrier_init();
   }
   __syncthreads();
+  if (threadIdx.x == 0) {
+    mbar_arrive_expect_tx(&bar_ld, bytes);
+    bulk_load(sS, S + (bh * nB + row0) * (long long)ldS, bytes, &bar_ld);
+  }
+  if (__syncthreads_and(mbar_wait(&bar_ld, 0, &never_abort, limit_ns)) == 0) {
+    // the copy did not land in time: wait (bounded) for it before the CTA exits
+    if (threadIdx.x == 0) {
+      report_error(-6);
+      mbar_wait(&bar_ld, 0, &never_abort, limit_ns);
+    }
+    return;
+  }
   const int warp = threadIdx.x >> 5;
   const int nW = (nB + 31) >> 5;
   for (int r = warp; r < nrows; r += kScoreWarps) {
