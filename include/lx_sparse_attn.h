@@ -117,6 +117,13 @@ lx_status lx_sparse_attn_plan(const lx_bhld* Q, const lx_bhld* K, double keep, l
 lx_status lx_quantize_qk(const lx_bhld* Q, const lx_bhld* K, int8_t* qc, float* qs, int8_t* kc, float* ks,
                          cudaStream_t stream);
 
+/* Steps a1 + a3 in one read of Q and K: the block means of lx_pool_means and
+ * the codes and scales of lx_quantize_qk, bit-identical to those two calls
+ * (all three run one kernel).  Arguments, layouts and errors as there; every
+ * output pointer must be non-NULL and 16-byte aligned. */
+lx_status lx_pool_quantize_qk(const lx_bhld* Q, const lx_bhld* K, float* mq, float* mk, int8_t* qc, float* qs,
+                              int8_t* kc, float* ks, cudaStream_t stream);
+
 /* Step a3 -- FP8 E4M3 V ("600倍加速…", §高效推理算子: "V FP8").
  * vc: uint8 [B,H,L,D] contiguous E4M3 codes; vs: fp32 [B,H,D] scales =
  * absmax over all L tokens / 448 (1 for an all-zero channel);

@@ -90,6 +90,16 @@ def test_host_argument_errors_before_launch(lib):
     other = _view(L=999)
     assert lib.lx_pool_means(ctypes.byref(q), ctypes.byref(other), 0x20000, 0x30000, s) == _abi.LX_ERR_INVALID
     assert lib.lx_pool_means(None, ctypes.byref(q), 0x20000, 0x30000, s) == _abi.LX_ERR_INVALID
+    # the fused means + codes pass: every output required, each 16-byte aligned
+    outs = [0x20000, 0x30000, 0x40000, 0x50000, 0x60000, 0x70000]
+    for i in range(6):
+        missing = list(outs)
+        missing[i] = None
+        assert lib.lx_pool_quantize_qk(ctypes.byref(q), ctypes.byref(q), *missing, s) == _abi.LX_ERR_INVALID
+        odd = list(outs)
+        odd[i] += 8
+        assert lib.lx_pool_quantize_qk(ctypes.byref(q), ctypes.byref(q), *odd, s) == _abi.LX_ERR_ALIGN
+    assert lib.lx_pool_quantize_qk(ctypes.byref(d96), ctypes.byref(d96), *outs, s) == _abi.LX_ERR_UNSUPPORTED
     # planner without enough workspace
     plan = _abi.LxPlan(0x40000, 0, 0, 0, 0, 0, 0, 0)
     assert lib.lx_sparse_attn_plan(ctypes.byref(q), ctypes.byref(q), 0.25, ctypes.byref(plan), 0x50000, 16, s) \

@@ -147,6 +147,26 @@ def lx_quantize_qk(Q, K, out=None, stream=None):
     return out
 
 
+def lx_pool_quantize_qk(Q, K, out=None, stream=None):
+    """Block means and INT8 codes of Q and K in one pass: (mq, mk, qc, qs, kc, ks)."""
+    lib = _abi.load()
+    B, H, L, D = Q.shape
+    nB = (L + LX_BLOCK - 1) // LX_BLOCK
+    if out is None:
+        dev = Q.device
+        out = (torch.empty((B, H, nB, D), dtype=torch.float32, device=dev),
+               torch.empty((B, H, nB, D), dtype=torch.float32, device=dev),
+               torch.empty((B, H, L, D), dtype=torch.int8, device=dev),
+               torch.empty((B, H, nB), dtype=torch.float32, device=dev),
+               torch.empty((B, H, L, D), dtype=torch.int8, device=dev),
+               torch.empty((B, H, nB), dtype=torch.float32, device=dev))
+    mq, mk, qc, qs, kc, ks = out
+    q, k = bhld(Q), bhld(K)
+    _check(lib.lx_pool_quantize_qk(ctypes.byref(q), ctypes.byref(k), _ptr(mq), _ptr(mk), _ptr(qc), _ptr(qs), _ptr(kc),
+                                   _ptr(ks), _stream(stream)), "lx_pool_quantize_qk")
+    return out
+
+
 def lx_quantize_v(V, out=None, amax_ws=None, stream=None):
     lib = _abi.load()
     B, H, L, D = V.shape

@@ -41,6 +41,7 @@ SIGNATURES = {
     "lx_score_topk": [_vp, _vp, _c_i64, _c_i64, _c_i64, _c_i64, _dbl, _P(LxPlan), _vp, _c_sz, _vp],
     "lx_sparse_attn_plan": [_P(LxBhld), _P(LxBhld), _dbl, _P(LxPlan), _vp, _c_sz, _vp],
     "lx_quantize_qk": [_P(LxBhld), _P(LxBhld), _vp, _vp, _vp, _vp, _vp],
+    "lx_pool_quantize_qk": [_P(LxBhld), _P(LxBhld), _vp, _vp, _vp, _vp, _vp, _vp, _vp],
     "lx_quantize_v": [_P(LxBhld), _vp, _vp, _vp, _vp],
     "lx_quantize_v_noalloc": [_P(LxBhld), _vp, _vp, _vp],
     "lx_attn_bf16": [_P(LxBhld), _P(LxBhld), _P(LxBhld), _P(LxPlan), _P(LxBhld), _vp],

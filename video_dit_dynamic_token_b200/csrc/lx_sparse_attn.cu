@@ -16,7 +16,8 @@
 namespace {
 
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;  // bound on every device-side wait
-constexpr int64_t kMaxPlannerNB = 2176;                       // score rows of 16 x nB fp32 in shared memory
+constexpr int64_t kMaxPlannerNB = 2176;  // selection: 8 score rows of nB fp32 in shared memory, 17 chunks of 128
+static_assert(kMaxPlannerNB <= 128 * lx::kMaxChunks, "selection chunk registers too few for the longest row");
 
 inline bool al16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 inline int64_t n_blocks(int64_t L) { return (L + LX_BLOCK - 1) / LX_BLOCK; }
@@ -112,11 +113,17 @@ bool make_map(CUtensorMap* m, const void* ptr, CUtensorMapDataType dt, int esz, 
 
 // ---------------------------------------------------------------- launchers
 template <int D>
-lx_status launch_pool(const lx_bhld* Q, const lx_bhld* K, float* mq, float* mk, cudaStream_t s) {
+lx_status launch_qk_pass(const lx_bhld* Q, const lx_bhld* K, float* mq, float* mk, int8_t* qc, float* qs, int8_t* kc,
+                         float* ks, cudaStream_t s) {
   const int64_t nB = n_blocks(Q->L);
-  const long long units = (long long)(Q->B * Q->H * nB);
-  dim3 grid((unsigned)((units + 7) / 8), 2);
-  lx::pool_means_kernel<D><<<grid, 256, 0, s>>>(view(Q), view(K), mq, mk, (int)Q->H, (int)Q->L, (int)nB, units);
+  dim3 grid((unsigned)(Q->B * Q->H * nB), 2);
+  const int H = (int)Q->H, L = (int)Q->L;
+  if (mq && qc)
+    lx::qk_block_pass_kernel<D, true, true><<<grid, 128, 0, s>>>(view(Q), view(K), mq, mk, qc, kc, qs, ks, H, L, (int)nB);
+  else if (mq)
+    lx::qk_block_pass_kernel<D, true, false><<<grid, 128, 0, s>>>(view(Q), view(K), mq, mk, qc, kc, qs, ks, H, L, (int)nB);
+  else
+    lx::qk_block_pass_kernel<D, false, true><<<grid, 128, 0, s>>>(view(Q), view(K), mq, mk, qc, kc, qs, ks, H, L, (int)nB);
   return launch_status();
 }
 
@@ -139,7 +146,7 @@ lx_status launch_score(const float* mq, const float* mk, int64_t BH, int64_t nB,
   if (cudaGetLastError() != cudaSuccess) return LX_ERR_CUDA;
   // selection: 8 rows per CTA, one warp per row
   const size_t smem = sizeof(float) * ((size_t)lx::kScoreRows * ldS +
-                                       lx::kScoreWarps * (256 + 2 * lx::kCandCap + ldS / 32));
+                                       lx::kScoreWarps * (lx::kBuckets + 2 * lx::kCandCap + ldS / 32));
   if (smem > 227 * 1024) return LX_ERR_UNSUPPORTED;
   if (cudaFuncSetAttribute(lx::select_topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
       cudaSuccess)
@@ -147,15 +154,6 @@ lx_status launch_score(const float* mq, const float* mk, int64_t BH, int64_t nB,
   dim3 grid((unsigned)((nB + lx::kScoreRows - 1) / lx::kScoreRows), (unsigned)BH);
   lx::select_topk_kernel<<<grid, 32 * lx::kScoreWarps, smem, s>>>(scores, (int)nB, (int)k, plan->idx, plan->mask,
                                                                    ldS, kWaitLimitNs);
-  return launch_status();
-}
-
-template <int D>
-lx_status launch_quant_qk(const lx_bhld* Q, const lx_bhld* K, int8_t* qc, float* qs, int8_t* kc, float* ks,
-                          cudaStream_t s) {
-  const int64_t nB = n_blocks(Q->L);
-  dim3 grid((unsigned)(Q->B * Q->H * nB), 2);
-  lx::quant_qk_kernel<D><<<grid, 128, 0, s>>>(view(Q), view(K), qc, kc, qs, ks, (int)Q->H, (int)Q->L, (int)nB);
   return launch_status();
 }
 
@@ -284,7 +282,8 @@ lx_status lx_pool_means(const lx_bhld* Q, const lx_bhld* K, float* mq, float* mk
   if ((st = check_bhld(Q)) != LX_OK || (st = check_bhld(K)) != LX_OK) return st;
   if (!same_shape(Q, K) || !mq || !mk) return LX_ERR_INVALID;
   if (!al16(mq) || !al16(mk)) return LX_ERR_ALIGN;
-  return Q->D == 128 ? launch_pool<128>(Q, K, mq, mk, stream) : launch_pool<64>(Q, K, mq, mk, stream);
+  return Q->D == 128 ? launch_qk_pass<128>(Q, K, mq, mk, nullptr, nullptr, nullptr, nullptr, stream)
+                     : launch_qk_pass<64>(Q, K, mq, mk, nullptr, nullptr, nullptr, nullptr, stream);
 }
 
 lx_status lx_score_topk(const float* mq, const float* mk, int64_t B, int64_t H, int64_t L, int64_t D, double keep,
@@ -334,8 +333,18 @@ lx_status lx_quantize_qk(const lx_bhld* Q, const lx_bhld* K, int8_t* qc, float* 
   if ((st = check_bhld(Q)) != LX_OK || (st = check_bhld(K)) != LX_OK) return st;
   if (!same_shape(Q, K) || !qc || !qs || !kc || !ks) return LX_ERR_INVALID;
   if (!al16(qc) || !al16(kc) || !al16(qs) || !al16(ks)) return LX_ERR_ALIGN;
-  return Q->D == 128 ? launch_quant_qk<128>(Q, K, qc, qs, kc, ks, stream)
-                     : launch_quant_qk<64>(Q, K, qc, qs, kc, ks, stream);
+  return Q->D == 128 ? launch_qk_pass<128>(Q, K, nullptr, nullptr, qc, qs, kc, ks, stream)
+                     : launch_qk_pass<64>(Q, K, nullptr, nullptr, qc, qs, kc, ks, stream);
+}
+
+lx_status lx_pool_quantize_qk(const lx_bhld* Q, const lx_bhld* K, float* mq, float* mk, int8_t* qc, float* qs,
+                              int8_t* kc, float* ks, cudaStream_t stream) {
+  lx_status st;
+  if ((st = check_bhld(Q)) != LX_OK || (st = check_bhld(K)) != LX_OK) return st;
+  if (!same_shape(Q, K) || !mq || !mk || !qc || !qs || !kc || !ks) return LX_ERR_INVALID;
+  if (!al16(mq) || !al16(mk) || !al16(qc) || !al16(kc) || !al16(qs) || !al16(ks)) return LX_ERR_ALIGN;
+  return Q->D == 128 ? launch_qk_pass<128>(Q, K, mq, mk, qc, qs, kc, ks, stream)
+                     : launch_qk_pass<64>(Q, K, mq, mk, qc, qs, kc, ks, stream);
 }
 
 lx_status lx_quantize_v(const lx_bhld* V, uint8_t* vc, float* vs, uint32_t* amax_ws, cudaStream_t stream) {

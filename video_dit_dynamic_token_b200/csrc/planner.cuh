@@ -38,55 +38,6 @@ __device__ __forceinline__ void acc_bf16x8(float (&a)[8], const uint4& v) {
 }
 
 // ---------------------------------------------------------------------------
-// a1: one warp per (tensor, b*h, block).  Lanes split a row into 16-byte chunks
-// (D/8 lanes per row); the warp walks the block's valid rows with 128-bit
-// streaming loads, accumulates in fp32, folds the lanes that share a chunk and
-// divides by the number of valid tokens.  Output fp32 [B*H, nB, D].
-template <int D>
-__global__ void __launch_bounds__(256) pool_means_kernel(BhldView q, BhldView k, float* __restrict__ mq,
-                                                        float* __restrict__ mk, int H, int L, int nB,
-                                                        long long units) {
-  constexpr int CH = D / 8;          // 16-byte chunks per row
-  constexpr int RPI = 32 / CH;       // rows per warp iteration
-  constexpr int ITERS = kBlock / RPI;
-  constexpr int UNROLL = 8;
-  const long long unit = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
-  if (unit >= units) return;
-  const int lane = threadIdx.x & 31;
-  const BhldView X = blockIdx.y == 0 ? q : k;
-  float* __restrict__ M = blockIdx.y == 0 ? mq : mk;
-  const long long bh = unit / nB;
-  const int blk = (int)(unit - bh * nB);
-  const long long b = bh / H, h = bh - b * H;
-  const int t0 = blk * kBlock;
-  const int cnt = min(kBlock, L - t0);
-  const int c = lane % CH, ro = lane / CH;
-  const __nv_bfloat16* base = X.p + b * X.sB + h * X.sH + (long long)t0 * X.sL + c * 8;
-  float a[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-#pragma unroll 1
-  for (int it0 = 0; it0 < ITERS; it0 += UNROLL) {
-    uint4 v[UNROLL];
-#pragma unroll
-    for (int u = 0; u < UNROLL; ++u) {
-      const int row = (it0 + u) * RPI + ro;
-      v[u] = row < cnt ? ld_stream_v4(base + (long long)row * X.sL) : make_uint4(0, 0, 0, 0);
-    }
-#pragma unroll
-    for (int u = 0; u < UNROLL; ++u) acc_bf16x8(a, v[u]);
-  }
-#pragma unroll
-  for (int off = CH; off < 32; off <<= 1)
-#pragma unroll
-    for (int i = 0; i < 8; ++i) a[i] += __shfl_xor_sync(0xffffffffu, a[i], off);
-  if (ro == 0) {
-    const float n = (float)cnt;
-    float4* out = reinterpret_cast<float4*>(M + (bh * nB + blk) * D + c * 8);
-    out[0] = make_float4(__fdiv_rn(a[0], n), __fdiv_rn(a[1], n), __fdiv_rn(a[2], n), __fdiv_rn(a[3], n));
-    out[1] = make_float4(__fdiv_rn(a[4], n), __fdiv_rn(a[5], n), __fdiv_rn(a[6], n), __fdiv_rn(a[7], n));
-  }
-}
-
-// ---------------------------------------------------------------------------
 // a2, scores: S[b,h,i,j] = Mq[b,h,i,:] . Mk[b,h,j,:] for all block pairs of a
 // head, on the tensor cores with fp32-level accuracy.  One 128-thread CTA
 // computes a 128-row x 128-key tile.  Each 32-dimension chunk of the pooled
@@ -236,14 +187,16 @@ __global__ void __launch_bounds__(128, 2) score_gemm_kernel(const __grid_constan
 // ---------------------------------------------------------------------------
 // a2, selection: one 256-thread CTA per (b*h, 8 query-block rows); the 8
 // score rows (contiguous in the workspace, ldS floats apart) arrive in shared
-// memory by one bulk copy, and each warp selects one row: scores are bucketed into 256 monotone buckets between
-// the row min and max; the bucket holding the k-th largest is resolved
-// exactly by ranking its members with the (score desc, index asc) order; the
-// kept ids are emitted in ascending order with a ballot scan that also yields
-// the bitmask words.
+// memory by one bulk copy, and each warp selects one row: scores are bucketed
+// into 128 monotone buckets between the row min and max; the bucket holding
+// the k-th largest is resolved exactly by ranking its members with the (score
+// desc, index asc) order; the kept ids are emitted in ascending order with
+// ballots that are also the bitmask words.
 constexpr int kScoreRows = 8;
 constexpr int kCandCap = 64;
 constexpr int kScoreWarps = 8;
+constexpr int kBuckets = 128;
+constexpr int kMaxChunks = 17;  // 128-score chunks of the longest row (nB <= 2176)
 
 __device__ __forceinline__ uint32_t lanemask_lt() {
   uint32_t m;
@@ -251,22 +204,55 @@ __device__ __forceinline__ uint32_t lanemask_lt() {
   return m;
 }
 
-__device__ __forceinline__ int score_bucket(float s, float mn, float scale) {
-  float t = (s - mn) * scale;
-  int b = (int)t;  // t >= 0 for finite s >= mn; NaN converts to 0
-  return min(255, max(0, b));
+// Bucket of a score: (s - mn) * scale clamped to [0, 127] and rounded to the
+// nearest integer by adding 1.5 * 2^23 (whose float spacing is 1), then read
+// from the bits.  Non-decreasing in s.  For a finite row s - mn >= 0; a NaN
+// (from a NaN or infinite score) clamps to 127, so the id is always in range.
+__device__ __forceinline__ uint32_t score_bucket(float s, float mn, float scale) {
+  const float t = fminf((s - mn) * scale, 127.0f);
+  return (__float_as_uint(t + 12582912.0f) - 0x4B400000u) & 127u;
 }
+
+// Four bucket ids packed one per byte (bit 7 of each byte clear): bit 7 of
+// byte e of the result is set where id_e > y (y + 1 <= 128, so no byte borrows
+// from its neighbour), or where id_e >= y for ge.
+__device__ __forceinline__ uint32_t bytes_gt(uint32_t pk, uint32_t y) {
+  return ((pk | 0x80808080u) - (y + 1u) * 0x01010101u) & 0x80808080u;
+}
+__device__ __forceinline__ uint32_t bytes_ge(uint32_t pk, uint32_t y) {
+  return ((pk | 0x80808080u) - y * 0x01010101u) & 0x80808080u;
+}
+// Bit 7 of byte e -> bit e (the four products land on bits 28..31 and
+// nowhere else below 32).
+__device__ __forceinline__ uint32_t high_bits_to_nibble(uint32_t m) { return ((m >> 7) * 0x10204080u) >> 28; }
 
 // Select the k best keys of one score row (warp-wide) and write the ascending
 // ids (and the bitmask words when `mask` is not null).  Returns the number of
-// ids written (k unless the row holds non-finite scores).
-__device__ int select_row(const float* __restrict__ s, int nB, int k, int* hist, float* cand_s, int* cand_j,
-                          uint32_t* selbits, int32_t* __restrict__ idx_out, uint32_t* __restrict__ mask_out) {
+// ids selected (k unless the row holds non-finite scores).  The row is walked
+// in chunks of 128 scores; lane l holds scores j = 128c + 32e + l (e = 0..3),
+// so that one ballot per e is one 32-bit mask word.  The histogram pass keeps
+// the four bucket ids of each lane and chunk in a register (pk[c]); the chunk
+// loops are unrolled to kMaxChunks so that pk stays in registers.  The ids are
+// gathered in the row's own shared buffer (no longer read once the ranking is
+// done) and the mask words in `selbits`, and both leave in coalesced stores.
+__device__ int select_row(float* s, int nB, int k, int* hist, float* cand_s, int* cand_j, uint32_t* selbits,
+                          int32_t* __restrict__ idx_out, uint32_t* __restrict__ mask_out) {
   const int lane = threadIdx.x & 31;
+  const int nC = (nB + 127) >> 7;
+  __syncwarp();
   float mn = INFINITY, mx = -INFINITY;
-  for (int j = lane; j < nB; j += 32) {
-    mn = fminf(mn, s[j]);
-    mx = fmaxf(mx, s[j]);
+  for (int ch = 0; ch < nC; ++ch) {
+    const int j0 = 128 * ch + 4 * lane;
+    if (j0 + 4 <= nB) {
+      const float4 v = *reinterpret_cast<const float4*>(s + j0);
+      mn = fminf(mn, fminf(fminf(v.x, v.y), fminf(v.z, v.w)));
+      mx = fmaxf(mx, fmaxf(fmaxf(v.x, v.y), fmaxf(v.z, v.w)));
+    } else {
+      for (int j = j0; j < nB; ++j) {
+        mn = fminf(mn, s[j]);
+        mx = fmaxf(mx, s[j]);
+      }
+    }
   }
 #pragma unroll
   for (int off = 16; off; off >>= 1) {
@@ -275,20 +261,37 @@ __device__ int select_row(const float* __restrict__ s, int nB, int k, int* hist,
   }
   const int nW = (nB + 31) >> 5;
   for (int w = lane; w < nW; w += 32) selbits[w] = 0u;
-  int bt = 0, need = k;
-  float scale = 0.f;
+  uint32_t bt = 0;
+  int need = k;
+  uint32_t pk[kMaxChunks];
+#pragma unroll
+  for (int ch = 0; ch < kMaxChunks; ++ch) pk[ch] = 0u;
   const bool flat = !(mx > mn);  // all equal (or non-finite): lowest ids win
   if (!flat) {
-    scale = 255.99f / (mx - mn);
-    for (int i = lane; i < 256; i += 32) hist[i] = 0;
+    const float scale = 127.99f / (mx - mn);
+    for (int i = lane; i < kBuckets; i += 32) hist[i] = 0;
     __syncwarp();
-    for (int j = lane; j < nB; j += 32) atomicAdd(&hist[score_bucket(s[j], mn, scale)], 1);
-    __syncwarp();
-    // lane l owns buckets 255-8l .. 248-8l (descending); find the bucket holding rank k
-    int cnt[8], tot = 0;
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      cnt[i] = hist[255 - 8 * lane - i];
+    for (int ch = 0; ch < kMaxChunks; ++ch) {
+      if (ch >= nC) break;
+      const int rem = nB - 128 * ch - lane;  // score e of this lane exists while 32e < rem
+      uint32_t p = 0;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        if (32 * e < rem) {
+          const uint32_t b = score_bucket(s[128 * ch + 32 * e + lane], mn, scale);
+          atomicAdd(&hist[b], 1);
+          p |= b << (8 * e);
+        }
+      }
+      pk[ch] = p;
+    }
+    __syncwarp();
+    // lane l owns buckets 127-4l .. 124-4l (descending); find the bucket holding rank k
+    int cnt[4], tot = 0;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      cnt[i] = hist[kBuckets - 1 - 4 * lane - i];
       tot += cnt[i];
     }
     int incl = tot;
@@ -305,10 +308,10 @@ __device__ int select_row(const float* __restrict__ s, int nB, int k, int* hist,
     if (lane == owner) {
       int above = excl;
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
+      for (int i = 0; i < 4; ++i) {
         if (my_bt < 0) {
           if (above + cnt[i] >= k) {
-            my_bt = 255 - 8 * lane - i;
+            my_bt = kBuckets - 1 - 4 * lane - i;
             my_need = k - above;
           } else {
             above += cnt[i];
@@ -316,22 +319,30 @@ __device__ int select_row(const float* __restrict__ s, int nB, int k, int* hist,
         }
       }
     }
-    bt = __shfl_sync(0xffffffffu, my_bt, owner);
+    bt = (uint32_t)__shfl_sync(0xffffffffu, my_bt, owner);
     need = __shfl_sync(0xffffffffu, my_need, owner);
     // members of bucket bt, ranked by (score desc, index asc)
     const int c = hist[bt];
     if (c <= kCandCap) {
+      const uint32_t lt = lanemask_lt();
       int base = 0;
-      for (int j0 = 0; j0 < nB; j0 += 32) {
-        const int j = j0 + lane;
-        const bool in = j < nB && score_bucket(s[j], mn, scale) == bt;
-        const uint32_t bal = __ballot_sync(0xffffffffu, in);
-        if (in) {
-          const int pos = base + __popc(bal & lanemask_lt());
-          cand_s[pos] = s[j];
-          cand_j[pos] = j;
+#pragma unroll
+      for (int ch = 0; ch < kMaxChunks; ++ch) {
+        if (ch >= nC) break;
+        const int rem = nB - 128 * ch - lane;
+        const uint32_t valid = (1u << (rem <= 0 ? 0 : min(4, (rem + 31) >> 5))) - 1u;
+        const uint32_t m = high_bits_to_nibble(bytes_ge(pk[ch], bt) & ~bytes_gt(pk[ch], bt)) & valid;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const uint32_t b = __ballot_sync(0xffffffffu, (m >> e) & 1u);
+          if ((m >> e) & 1u) {
+            const int pos = base + __popc(b & lt);
+            const int j = 128 * ch + 32 * e + lane;
+            cand_s[pos] = s[j];
+            cand_j[pos] = j;
+          }
+          base += __popc(b);
         }
-        base += __popc(bal);
       }
       __syncwarp();
       for (int i = lane; i < c; i += 32) {
@@ -367,25 +378,51 @@ __device__ int select_row(const float* __restrict__ s, int nB, int k, int* hist,
     }
     __syncwarp();
   }
-  // emit ascending ids
+  // emit ascending ids into the row buffer; mask word 4c + e is the ballot of
+  // score e of the lanes and replaces selbits word 4c + e once it has been read
+  int* ids = reinterpret_cast<int*>(s);
+  const uint32_t lt = lanemask_lt();
   int written = 0;
-  for (int j0 = 0; j0 < nB; j0 += 32) {
-    const int j = j0 + lane;
-    bool sel = false;
-    if (j < nB) {
-      if (flat)
-        sel = j < k;
-      else {
-        const int bk = score_bucket(s[j], mn, scale);
-        sel = bk > bt || (bk == bt && ((selbits[j >> 5] >> (j & 31)) & 1u));
+#pragma unroll
+  for (int ch = 0; ch < kMaxChunks; ++ch) {
+    if (ch >= nC) break;
+    const int rem = nB - 128 * ch - lane;
+    const int ne = rem <= 0 ? 0 : min(4, (rem + 31) >> 5);  // scores of this lane in the chunk
+    const uint32_t valid = (1u << ne) - 1u;
+    uint32_t sel;
+    if (flat) {
+      const int remk = min(k, nB) - 128 * ch - lane;
+      sel = (1u << (remk <= 0 ? 0 : min(4, (remk + 31) >> 5))) - 1u;
+    } else {
+      const uint32_t gt = bytes_gt(pk[ch], bt);
+      sel = high_bits_to_nibble(gt) & valid;
+      uint32_t eq = high_bits_to_nibble(bytes_ge(pk[ch], bt) & ~gt) & valid;
+      while (eq) {
+        const int e = __ffs(eq) - 1;
+        eq &= eq - 1;
+        sel |= ((selbits[4 * ch + e] >> lane) & 1u) << e;
       }
     }
-    const uint32_t bal = __ballot_sync(0xffffffffu, sel);
-    const int pos = written + __popc(bal & lanemask_lt());
-    if (sel && pos < k) idx_out[pos] = j;
-    if (mask_out && lane == 0) mask_out[j0 >> 5] = bal;
-    written += __popc(bal);
+    const uint32_t b0 = __ballot_sync(0xffffffffu, sel & 1u), b1 = __ballot_sync(0xffffffffu, sel & 2u);
+    const uint32_t b2 = __ballot_sync(0xffffffffu, sel & 4u), b3 = __ballot_sync(0xffffffffu, sel & 8u);
+    const int p0 = __popc(b0), p1 = __popc(b1), p2 = __popc(b2);
+    const int j = 128 * ch + lane;
+    if (sel) {
+      int pos;
+      if ((sel & 1u) && (pos = written + __popc(b0 & lt)) < k) ids[pos] = j;
+      if ((sel & 2u) && (pos = written + p0 + __popc(b1 & lt)) < k) ids[pos] = j + 32;
+      if ((sel & 4u) && (pos = written + p0 + p1 + __popc(b2 & lt)) < k) ids[pos] = j + 64;
+      if ((sel & 8u) && (pos = written + p0 + p1 + p2 + __popc(b3 & lt)) < k) ids[pos] = j + 96;
+    }
+    // every lane's selbits reads for this chunk fed the ballots above
+    if (lane < 4 && 4 * ch + lane < nW) selbits[4 * ch + lane] = lane == 0 ? b0 : (lane == 1 ? b1 : (lane == 2 ? b2 : b3));
+    written += p0 + p1 + p2 + __popc(b3);
   }
+  __syncwarp();
+  const int n_out = min(written, k);
+  for (int i = lane; i < n_out; i += 32) idx_out[i] = ids[i];
+  if (mask_out)
+    for (int w = lane; w < nW; w += 32) mask_out[w] = selbits[w];
   return written;
 }
 
@@ -395,8 +432,8 @@ __global__ void __launch_bounds__(32 * kScoreWarps) select_topk_kernel(const flo
                                                                       unsigned long long limit_ns) {
   extern __shared__ __align__(16) float smem_f[];
   float* sS = smem_f;                                                        // [8][ldS]
-  int* hist = reinterpret_cast<int*>(sS + kScoreRows * ldS);                 // warps x 256
-  float* cand_s = reinterpret_cast<float*>(hist + kScoreWarps * 256);       // warps x 64
+  int* hist = reinterpret_cast<int*>(sS + kScoreRows * ldS);                 // warps x 128
+  float* cand_s = reinterpret_cast<float*>(hist + kScoreWarps * kBuckets);  // warps x 64
   int* cand_j = reinterpret_cast<int*>(cand_s + kScoreWarps * kCandCap);    // warps x 64
   uint32_t* selbits = reinterpret_cast<uint32_t*>(cand_j + kScoreWarps * kCandCap);  // warps x ldS/32
   __shared__ uint64_t bar_ld;
@@ -416,7 +453,12 @@ __global__ void __launch_bounds__(32 * kScoreWarps) select_topk_kernel(const flo
     mbar_arrive_expect_tx(&bar_ld, bytes);
     bulk_load(sS, S + (bh * nB + row0) * (long long)ldS, bytes, &bar_ld);
   }
-  if (__syncthreads_and(mbar_wait(&bar_ld, 0, &never_abort, limit_ns)) == 0) {
+  // one thread waits (suspending between polls, so that the waiting CTA takes
+  // no issue slots from the CTAs that compute); after the barrier every thread
+  // observes the completed phase itself, which makes the copied rows visible to it
+  bool landed = true;
+  if (threadIdx.x == 0) landed = mbar_wait_hint(&bar_ld, 0, &never_abort, limit_ns, 20000u);
+  if (__syncthreads_and(landed) == 0) {
     // the copy did not land in time: wait (bounded) for it before the CTA exits
     if (threadIdx.x == 0) {
       report_error(-6);
@@ -424,13 +466,14 @@ __global__ void __launch_bounds__(32 * kScoreWarps) select_topk_kernel(const flo
     }
     return;
   }
+  if (!mbar_try_wait(&bar_ld, 0)) report_error(-6);  // cannot fail: the phase has completed
   const int warp = threadIdx.x >> 5;
   const int nW = (nB + 31) >> 5;
   for (int r = warp; r < nrows; r += kScoreWarps) {
     const long long row = bh * nB + row0 + r;
-    const int got = select_row(sS + r * ldS, nB, k, hist + warp * 256, cand_s + warp * kCandCap,
-                               cand_j + warp * kCandCap, selbits + warp * (ldS / 32), idx + row * k,
-                               mask ? mask + row * nW : nullptr);
+    const int got = select_row(sS + r * ldS, nB, k, hist + warp * kBuckets, cand_s + warp * kCandCap,
+                               cand_j + warp * kCandCap, selbits + warp * (ldS / 32),
+                               idx + row * k, mask ? mask + row * nW : nullptr);
     if (got != k && (threadIdx.x & 31) == 0) {
       report_error(-7);  // non-finite scores: the row could not be ordered
       for (int p = got; p < k; ++p) idx[row * k + p] = -1;

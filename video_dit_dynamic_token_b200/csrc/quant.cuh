@@ -41,58 +41,93 @@ __device__ __forceinline__ uint32_t e4m3x4(float a, float b, float c, float d) {
 }
 
 // ---------------------------------------------------------------------------
-// Q/K: one 128-thread CTA per (tensor, b*h, block).  Thread t covers row t/2,
-// half (t&1) of the D channels (D/2 values = D/16 16-byte chunks).
-template <int D>
-__global__ void __launch_bounds__(128) quant_qk_kernel(BhldView q, BhldView k, int8_t* __restrict__ qc,
-                                                      int8_t* __restrict__ kc, float* __restrict__ qs,
-                                                      float* __restrict__ ks, int H, int L, int nB) {
-  constexpr int NCH = D / 16;  // 16-byte input chunks per thread
+// Q/K block pass (steps a1 and a3 in one read): one 128-thread CTA per
+// (tensor, b*h, 64-token block).  The D/8 16-byte chunks of a row go to
+// consecutive lanes (a warp loads whole rows, coalesced) and the 128/(D/8) row
+// groups of the CTA take rows r, r + RG, ...; every thread keeps its D/16 rows
+// of one chunk in registers.  MEANS: per-channel sums over the thread's rows,
+// then over the row groups in a fixed order (shuffles inside a warp, then the
+// four warps in shared memory), divided by the valid token count.  CODES: the
+// block absmax (max is exact in any order) gives inv = 127/a, and each value
+// becomes rint(x * inv) clamped to +-127; the scale a/127 (1 for an all-zero
+// block) is stored per block.  Either part may be switched off, so the pool,
+// the quantiser and the fused pass share one code path and agree bit for bit.
+template <int D, bool MEANS, bool CODES>
+__global__ void __launch_bounds__(128) qk_block_pass_kernel(BhldView q, BhldView k, float* __restrict__ mq,
+                                                           float* __restrict__ mk, int8_t* __restrict__ qc,
+                                                           int8_t* __restrict__ kc, float* __restrict__ qs,
+                                                           float* __restrict__ ks, int H, int L, int nB) {
+  constexpr int CH = D / 8;      // 16-byte chunks per row
+  constexpr int RG = 128 / CH;   // row groups in the CTA
+  constexpr int NR = kBlock / RG;  // rows per thread (= D/16)
   const BhldView X = blockIdx.y == 0 ? q : k;
-  int8_t* __restrict__ C = blockIdx.y == 0 ? qc : kc;
-  float* __restrict__ S = blockIdx.y == 0 ? qs : ks;
   const long long unit = blockIdx.x;
   const long long bh = unit / nB;
   const int blk = (int)(unit - bh * nB);
   const long long b = bh / H, h = bh - b * H;
   const int t0 = blk * kBlock;
   const int cnt = min(kBlock, L - t0);
-  const int row = threadIdx.x >> 1, col0 = (threadIdx.x & 1) * (D / 2);
-  uint4 v[NCH];
-  const __nv_bfloat16* src = X.p + b * X.sB + h * X.sH + (long long)(t0 + row) * X.sL + col0;
+  const int c = threadIdx.x % CH, r = threadIdx.x / CH;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const __nv_bfloat16* src = X.p + b * X.sB + h * X.sH + (long long)(t0 + r) * X.sL + c * 8;
+  uint4 v[NR];
 #pragma unroll
-  for (int i = 0; i < NCH; ++i) v[i] = row < cnt ? ld_stream_v4(src + 8 * i) : make_uint4(0, 0, 0, 0);
-  float a = 0.f;
-#pragma unroll
-  for (int i = 0; i < NCH; ++i) {
-    const uint32_t w[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
-#pragma unroll
-    for (int e = 0; e < 4; ++e) a = fmaxf(a, fmaxf(fabsf(bf16lo(w[e])), fabsf(bf16hi(w[e]))));
-  }
-#pragma unroll
-  for (int off = 16; off; off >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, off));
+  for (int i = 0; i < NR; ++i) v[i] = r + RG * i < cnt ? ld_stream_v4(src + (long long)(RG * i) * X.sL) : make_uint4(0, 0, 0, 0);
+  __shared__ float part[MEANS ? 4 : 1][MEANS ? D : 1];
   __shared__ float red[4];
-  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = a;
+  if constexpr (MEANS) {
+    float a[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int i = 0; i < NR; ++i) acc_bf16x8(a, v[i]);
+#pragma unroll
+    for (int off = CH; off < 32; off <<= 1)
+#pragma unroll
+      for (int e = 0; e < 8; ++e) a[e] += __shfl_xor_sync(0xffffffffu, a[e], off);
+    if (lane < CH)
+#pragma unroll
+      for (int e = 0; e < 8; ++e) part[warp][c * 8 + e] = a[e];
+  }
+  float amax = 0.f;
+  if constexpr (CODES) {
+#pragma unroll
+    for (int i = 0; i < NR; ++i) {
+      const uint32_t w[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) amax = fmaxf(amax, fmaxf(fabsf(bf16lo(w[e])), fabsf(bf16hi(w[e]))));
+    }
+#pragma unroll
+    for (int off = 16; off; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
+    if (lane == 0) red[warp] = amax;
+  }
   __syncthreads();
-  a = fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3]));
-  const float inv = a > 0.f ? __fdiv_rn(127.0f, a) : 0.f;
-  if (row < cnt) {
-    int8_t* dst = C + (bh * L + t0 + row) * D + col0;
-#pragma unroll
-    for (int i = 0; i < NCH; i += 2) {
-      uint32_t o[4];
-#pragma unroll
-      for (int hh = 0; hh < 2; ++hh) {
-        const uint32_t w[4] = {v[i + hh].x, v[i + hh].y, v[i + hh].z, v[i + hh].w};
-        o[2 * hh] = pack_i8x4(quant_i8(bf16lo(w[0]), inv), quant_i8(bf16hi(w[0]), inv), quant_i8(bf16lo(w[1]), inv),
-                              quant_i8(bf16hi(w[1]), inv));
-        o[2 * hh + 1] = pack_i8x4(quant_i8(bf16lo(w[2]), inv), quant_i8(bf16hi(w[2]), inv),
-                                  quant_i8(bf16lo(w[3]), inv), quant_i8(bf16hi(w[3]), inv));
-      }
-      *reinterpret_cast<uint4*>(dst + 8 * i) = make_uint4(o[0], o[1], o[2], o[3]);
+  if constexpr (MEANS) {
+    if (threadIdx.x < D) {
+      const float sum = ((part[0][threadIdx.x] + part[1][threadIdx.x]) + part[2][threadIdx.x]) + part[3][threadIdx.x];
+      float* __restrict__ M = blockIdx.y == 0 ? mq : mk;
+      M[(bh * nB + blk) * D + threadIdx.x] = __fdiv_rn(sum, (float)cnt);
     }
   }
-  if (threadIdx.x == 0) S[bh * nB + blk] = a > 0.f ? __fdiv_rn(a, 127.0f) : 1.0f;
+  if constexpr (CODES) {
+    amax = fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3]));
+    const float inv = amax > 0.f ? __fdiv_rn(127.0f, amax) : 0.f;
+    int8_t* __restrict__ C = blockIdx.y == 0 ? qc : kc;
+    int8_t* dst = C + (bh * L + t0 + r) * D + c * 8;
+#pragma unroll
+    for (int i = 0; i < NR; ++i) {
+      if (r + RG * i < cnt) {
+        const uint32_t w[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
+        const uint32_t o0 = pack_i8x4(quant_i8(bf16lo(w[0]), inv), quant_i8(bf16hi(w[0]), inv),
+                                      quant_i8(bf16lo(w[1]), inv), quant_i8(bf16hi(w[1]), inv));
+        const uint32_t o1 = pack_i8x4(quant_i8(bf16lo(w[2]), inv), quant_i8(bf16hi(w[2]), inv),
+                                      quant_i8(bf16lo(w[3]), inv), quant_i8(bf16hi(w[3]), inv));
+        *reinterpret_cast<uint2*>(dst + (long long)(RG * i) * D) = make_uint2(o0, o1);
+      }
+    }
+    if (threadIdx.x == 0) {
+      float* __restrict__ S = blockIdx.y == 0 ? qs : ks;
+      S[bh * nB + blk] = amax > 0.f ? __fdiv_rn(amax, 127.0f) : 1.0f;
+    }
+  }
 }
 
 template <int NCH>
