@@ -130,12 +130,6 @@ __global__ void __launch_bounds__(128) qk_block_pass_kernel(BhldView q, BhldView
   }
 }
 
-template <int NCH>
-__device__ __forceinline__ void load_row_half(const __nv_bfloat16* src, bool valid, uint4 (&v)[NCH]) {
-#pragma unroll
-  for (int i = 0; i < NCH; ++i) v[i] = valid ? ld_stream_v4(src + 8 * i) : make_uint4(0, 0, 0, 0);
-}
-
 // ---------------------------------------------------------------------------
 // V, pass 1: per-channel absmax.  One 128-thread CTA per (b*h, 512-token span);
 // lanes cover 16-byte channel chunks; the CTA folds its rows in shared memory
@@ -175,45 +169,55 @@ __global__ void __launch_bounds__(128) v_absmax_kernel(BhldView v, uint32_t* __r
   }
 }
 
-__device__ __forceinline__ const __nv_bfloat16* v_row_src(const BhldView& v, long long bh, int blk, int H, int row,
-                                                         int col0) {
-  const long long b = bh / H, h = bh - b * H;
-  return v.p + b * v.sB + h * v.sH + (long long)(blk * kBlock + row) * v.sL + col0;
-}
-
+// ---------------------------------------------------------------------------
 // V, pass 2: codes.  A unit is one (b*h, 64-token block); each persistent
-// 128-thread CTA walks a contiguous range of units, thread t covering row t/2
-// and half of the channels, with the next unit's rows loaded into a second
-// register set while the current one is converted.  The per-channel
-// reciprocal scales are rebuilt in shared memory when b*h changes; the CTA
-// that converts block 0 of a head also writes the head's channel scales.
+// 128-thread CTA walks a contiguous range of units.  As in the Q/K pass, the
+// D/8 16-byte chunks of a row go to consecutive lanes and thread t takes rows
+// r, r + RG, ... of chunk c = t mod (D/8), so a warp loads and stores whole
+// rows; the next unit's rows are loaded into a second register set while the
+// current one is converted.  A thread's 8 channels never change, so their
+// reciprocal scales live in registers and are rebuilt when b*h changes; the
+// CTA that converts block 0 of a head also writes the head's channel scales.
 template <int D>
 __global__ void __launch_bounds__(128, 4) v_quant_kernel(BhldView v, const uint32_t* __restrict__ amax,
                                                         uint8_t* __restrict__ vc, float* __restrict__ vs, int H,
                                                         int L, int nB, long long nunits, long long units_per_cta) {
-  constexpr int NCH = D / 16;
+  constexpr int CH = D / 8;        // 16-byte chunks per row
+  constexpr int RG = 128 / CH;     // row groups in the CTA
+  constexpr int NR = kBlock / RG;  // rows per thread
   const long long u_begin = (long long)blockIdx.x * units_per_cta;
   const long long u_end = min(u_begin + units_per_cta, nunits);
   if (u_begin >= u_end) return;
-  __shared__ float inv_s[D];
-  const int row = threadIdx.x >> 1, col0 = (threadIdx.x & 1) * (D / 2);
-  uint4 x[NCH], xn[NCH];
+  const int c = threadIdx.x % CH, r = threadIdx.x / CH;
+  uint4 x[NR], xn[NR];
   long long bh = u_begin / nB;
   int blk = (int)(u_begin - bh * nB);
-  load_row_half<NCH>(v_row_src(v, bh, blk, H, row, col0), row < min(kBlock, L - blk * kBlock), x);
-  long long bh_s = -1;  // head whose scales sit in inv_s
+  {
+    const long long b = bh / H, h = bh - b * H;
+    const __nv_bfloat16* src = v.p + b * v.sB + h * v.sH + (long long)(blk * kBlock + r) * v.sL + c * 8;
+    const int cnt = min(kBlock, L - blk * kBlock);
+#pragma unroll
+    for (int i = 0; i < NR; ++i) x[i] = r + RG * i < cnt ? ld_stream_v4(src + (long long)(RG * i) * v.sL) : make_uint4(0, 0, 0, 0);
+  }
+  long long bh_s = -1;  // head whose scales sit in inv
+  float inv[8];
   for (long long u = u_begin; u < u_end; ++u) {
     const long long bhn = (u + 1) / nB;
     const int blkn = (int)(u + 1 - bhn * nB);
-    if (u + 1 < u_end)
-      load_row_half<NCH>(v_row_src(v, bhn, blkn, H, row, col0), row < min(kBlock, L - blkn * kBlock), xn);
+    if (u + 1 < u_end) {
+      const long long b = bhn / H, h = bhn - b * H;
+      const __nv_bfloat16* src = v.p + b * v.sB + h * v.sH + (long long)(blkn * kBlock + r) * v.sL + c * 8;
+      const int cnt = min(kBlock, L - blkn * kBlock);
+#pragma unroll
+      for (int i = 0; i < NR; ++i)
+        xn[i] = r + RG * i < cnt ? ld_stream_v4(src + (long long)(RG * i) * v.sL) : make_uint4(0, 0, 0, 0);
+    }
     if (bh != bh_s) {
-      __syncthreads();  // every thread is done with the previous head's scales
-      for (int ch = threadIdx.x; ch < D; ch += blockDim.x) {
-        const float a = __uint_as_float(amax[bh * D + ch]);
-        inv_s[ch] = a > 0.f ? __fdiv_rn(448.0f, a) : 0.f;
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        const float a = __uint_as_float(amax[bh * D + c * 8 + e]);
+        inv[e] = a > 0.f ? __fdiv_rn(448.0f, a) : 0.f;
       }
-      __syncthreads();
       bh_s = bh;
     }
     if (blk == 0)
@@ -221,27 +225,21 @@ __global__ void __launch_bounds__(128, 4) v_quant_kernel(BhldView v, const uint3
         const float a = __uint_as_float(amax[bh * D + ch]);
         vs[bh * D + ch] = a > 0.f ? __fdiv_rn(a, 448.0f) : 1.0f;
       }
-    if (row < min(kBlock, L - blk * kBlock)) {
-      uint8_t* dst = vc + (bh * L + blk * kBlock + row) * D + col0;
+    const int cnt = min(kBlock, L - blk * kBlock);
+    uint8_t* dst = vc + (bh * L + blk * kBlock + r) * D + c * 8;
 #pragma unroll
-      for (int i = 0; i < NCH; i += 2) {
-        uint32_t o[4];
+    for (int i = 0; i < NR; ++i) {
+      if (r + RG * i < cnt) {
+        const uint32_t w[4] = {x[i].x, x[i].y, x[i].z, x[i].w};
+        uint32_t p[4];
 #pragma unroll
-        for (int hh = 0; hh < 2; ++hh) {
-          const uint32_t w[4] = {x[i + hh].x, x[i + hh].y, x[i + hh].z, x[i + hh].w};
-          const float* iv = inv_s + col0 + 8 * (i + hh);
-          uint32_t p[4];
-#pragma unroll
-          for (int e = 0; e < 4; ++e)
-            p[e] = e4m3x2(__fmul_rn(bf16lo(w[e]), iv[2 * e]), __fmul_rn(bf16hi(w[e]), iv[2 * e + 1]));
-          o[2 * hh] = p[0] | (p[1] << 16);
-          o[2 * hh + 1] = p[2] | (p[3] << 16);
-        }
-        *reinterpret_cast<uint4*>(dst + 8 * i) = make_uint4(o[0], o[1], o[2], o[3]);
+        for (int e = 0; e < 4; ++e)
+          p[e] = e4m3x2(__fmul_rn(bf16lo(w[e]), inv[2 * e]), __fmul_rn(bf16hi(w[e]), inv[2 * e + 1]));
+        *reinterpret_cast<uint2*>(dst + (long long)(RG * i) * D) = make_uint2(p[0] | (p[1] << 16), p[2] | (p[3] << 16));
       }
     }
 #pragma unroll
-    for (int i = 0; i < NCH; ++i) x[i] = xn[i];
+    for (int i = 0; i < NR; ++i) x[i] = xn[i];
     bh = bhn;
     blk = blkn;
   }
