@@ -16,13 +16,28 @@ namespace lx {
 __device__ __forceinline__ float bf16lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
 
-__device__ __forceinline__ uint32_t pack_i8x4(int a, int b, int c, int d) {
-  return (uint32_t)(a & 0xFF) | ((uint32_t)(b & 0xFF) << 8) | ((uint32_t)(c & 0xFF) << 16) | ((uint32_t)(d & 0xFF) << 24);
+// Bits of fl32(x * inv) + 1.5 * 2^23.  With |x| <= a and inv = fl32(127 / a),
+// |fl32(x * inv)| <= 127 (1 + 2^-24), so the sum lies in [2^23, 2^24) where
+// the float spacing is 1: the add rounds x * inv to the nearest integer, half
+// to even, and the low byte of the bits is that integer as a two's-complement
+// int8 in [-127, 127] (the +-127 clamp cannot bind).
+__device__ __forceinline__ uint32_t i8_code_bits(float x, float inv) {
+  return __float_as_uint(__fadd_rn(__fmul_rn(x, inv), 12582912.0f));
 }
-
-__device__ __forceinline__ int quant_i8(float x, float inv) {
-  const int q = __float2int_rn(__fmul_rn(x, inv));  // round half to even
-  return max(-127, min(127, q));
+// Low bytes of a, b, c, d packed into one word, a in the lowest byte.
+__device__ __forceinline__ uint32_t pack_low_bytes(uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+  return __byte_perm(__byte_perm(a, b, 0x0040), __byte_perm(c, d, 0x0040), 0x5410);
+}
+// The INT8 codes of the 8 bf16 values of one 16-byte chunk.
+__device__ __forceinline__ uint2 i8_codes_x8(const uint4& v, float inv) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+  uint32_t t[8];
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    t[2 * e] = i8_code_bits(bf16lo(w[e]), inv);
+    t[2 * e + 1] = i8_code_bits(bf16hi(w[e]), inv);
+  }
+  return make_uint2(pack_low_bytes(t[0], t[1], t[2], t[3]), pack_low_bytes(t[4], t[5], t[6], t[7]));
 }
 
 // Two fp32 values to two E4M3 codes (lo in bits 0..7), round to nearest even, saturating.
@@ -89,12 +104,16 @@ __global__ void __launch_bounds__(128) qk_block_pass_kernel(BhldView q, BhldView
   }
   float amax = 0.f;
   if constexpr (CODES) {
+    // |x| maxima on bf16 pairs (exact: widening to fp32 keeps order, and both
+    // maxima ignore a NaN operand as fmaxf does)
+    __nv_bfloat162 m2 = __floats2bfloat162_rn(0.f, 0.f);
 #pragma unroll
     for (int i = 0; i < NR; ++i) {
       const uint32_t w[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
 #pragma unroll
-      for (int e = 0; e < 4; ++e) amax = fmaxf(amax, fmaxf(fabsf(bf16lo(w[e])), fabsf(bf16hi(w[e]))));
+      for (int e = 0; e < 4; ++e) m2 = __hmax2(m2, __habs2(*reinterpret_cast<const __nv_bfloat162*>(&w[e])));
     }
+    amax = fmaxf(__low2float(m2), __high2float(m2));
 #pragma unroll
     for (int off = 16; off; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
     if (lane == 0) red[warp] = amax;
@@ -114,14 +133,7 @@ __global__ void __launch_bounds__(128) qk_block_pass_kernel(BhldView q, BhldView
     int8_t* dst = C + (bh * L + t0 + r) * D + c * 8;
 #pragma unroll
     for (int i = 0; i < NR; ++i) {
-      if (r + RG * i < cnt) {
-        const uint32_t w[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
-        const uint32_t o0 = pack_i8x4(quant_i8(bf16lo(w[0]), inv), quant_i8(bf16hi(w[0]), inv),
-                                      quant_i8(bf16lo(w[1]), inv), quant_i8(bf16hi(w[1]), inv));
-        const uint32_t o1 = pack_i8x4(quant_i8(bf16lo(w[2]), inv), quant_i8(bf16hi(w[2]), inv),
-                                      quant_i8(bf16lo(w[3]), inv), quant_i8(bf16hi(w[3]), inv));
-        *reinterpret_cast<uint2*>(dst + (long long)(RG * i) * D) = make_uint2(o0, o1);
-      }
+      if (r + RG * i < cnt) *reinterpret_cast<uint2*>(dst + (long long)(RG * i) * D) = i8_codes_x8(v[i], inv);
     }
     if (threadIdx.x == 0) {
       float* __restrict__ S = blockIdx.y == 0 ? qs : ks;
