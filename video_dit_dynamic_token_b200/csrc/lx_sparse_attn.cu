@@ -130,7 +130,7 @@ lx_status launch_qk_pass(const lx_bhld* Q, const lx_bhld* K, float* mq, float* m
 template <int D>
 lx_status launch_score(const float* mq, const float* mk, int64_t BH, int64_t nB, int64_t k, float* scores,
                        lx_plan* plan, cudaStream_t s) {
-  // scores: tf32 x3 tensor-core GEMM, one 128 x 256 tile per CTA
+  // scores: tf32 x3 tensor-core GEMM, one 128 x 128 tile per CTA
   CUtensorMap tq, tk;
   const auto f32 = CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
   if (!make_map(&tq, mq, f32, 4, 1, BH, nB, D, BH * nB * D, nB * D, D, lx::kSgK, lx::kSgM) ||

@@ -40,19 +40,20 @@ __device__ __forceinline__ void acc_bf16x8(float (&a)[8], const uint4& v) {
 // ---------------------------------------------------------------------------
 // a2, scores: S[b,h,i,j] = Mq[b,h,i,:] . Mk[b,h,j,:] for all block pairs of a
 // head, on the tensor cores with fp32-level accuracy.  One 128-thread CTA
-// computes a 128-row x 128-key tile.  Each 32-dimension chunk of the pooled
-// means arrives by TMA (fp32, 128-byte swizzle) into one of two chunk buffers
+// computes a 128-row x 128-key tile; 48 KB of shared memory and 128 TMEM
+// columns let four CTAs share an SM.  Each 16-dimension chunk of the pooled
+// means arrives by TMA (fp32, 64-byte swizzle) into one of two chunk buffers
 // (the next chunk loads while the current one is used) and is split in place
 // into a tf32-exact high part h = x rounded to 10 mantissa bits, plus the
-// remainder l = x - h (exact in fp32) in a third buffer; three kind::tf32 MMAs (h.h + h.l + l.h) then
-// accumulate in TMEM, leaving only the l.l term and the tf32 truncation of l,
+// remainder l = x - h (exact in fp32) in a third buffer; three kind::tf32
+// MMAs (h.h + h.l + l.h) then accumulate in TMEM, leaving only the l.l term and the tf32 truncation of l,
 // about 2^-22 of each product.  The tile leaves through shared memory, one
 // 128-byte row segment per warp store; rows are ldS = nB rounded up to 32
 // floats apart, so that each starts on a 128-byte boundary (columns nB..ldS-1
 // are never written).  Dividing by sqrt(d) changes no ranking and is left out.
-constexpr int kSgM = 128, kSgN = 128, kSgK = 32;  // rows, keys, dimensions per chunk
-constexpr int kSgA = kSgM * kSgK * 4;             // bytes of one A chunk (16 KB)
-constexpr int kSgB = kSgN * kSgK * 4;             // bytes of one B chunk (16 KB)
+constexpr int kSgM = 128, kSgN = 128, kSgK = 16;  // rows, keys, dimensions per chunk (64-byte rows)
+constexpr int kSgA = kSgM * kSgK * 4;             // bytes of one A chunk (8 KB)
+constexpr int kSgB = kSgN * kSgK * 4;             // bytes of one B chunk (8 KB)
 constexpr int kSgRaw = kSgA + kSgB;               // one raw chunk (A then B)
 constexpr int kSgSmem = 3 * kSgRaw;              // two chunk buffers (raw, then high part) + low parts
 constexpr uint32_t kSgIdesc = instr_desc(IDESC_DF32, IDESC_TF32, IDESC_TF32, 0, 0, kSgM, kSgN);
@@ -62,7 +63,7 @@ __device__ __forceinline__ float tf32_high(float v) {
 }
 
 template <int D>
-__global__ void __launch_bounds__(128, 2) score_gemm_kernel(const __grid_constant__ CUtensorMap tmQ,
+__global__ void __launch_bounds__(128, 4) score_gemm_kernel(const __grid_constant__ CUtensorMap tmQ,
                                                            const __grid_constant__ CUtensorMap tmK,
                                                            float* __restrict__ S, int nB, int ldS,
                                                            unsigned long long limit_ns) {
@@ -132,10 +133,10 @@ __global__ void __launch_bounds__(128, 2) score_gemm_kernel(const __grid_constan
       tc_fence_after();
 #pragma unroll
       for (int ks = 0; ks < kSgK / 8; ++ks) {  // 8 tf32 values = 32 bytes per MMA
-        const uint64_t ah = smem_desc(smem_u32(hi) + ks * 32, 16, 8 * 128, SW_128B);
-        const uint64_t al = smem_desc(smem_u32(lo) + ks * 32, 16, 8 * 128, SW_128B);
-        const uint64_t bhd = smem_desc(smem_u32(hi + kSgA) + ks * 32, 16, 8 * 128, SW_128B);
-        const uint64_t bld = smem_desc(smem_u32(lo + kSgA) + ks * 32, 16, 8 * 128, SW_128B);
+        const uint64_t ah = smem_desc(smem_u32(hi) + ks * 32, 16, 8 * 64, SW_64B);
+        const uint64_t al = smem_desc(smem_u32(lo) + ks * 32, 16, 8 * 64, SW_64B);
+        const uint64_t bhd = smem_desc(smem_u32(hi + kSgA) + ks * 32, 16, 8 * 64, SW_64B);
+        const uint64_t bld = smem_desc(smem_u32(lo + kSgA) + ks * 32, 16, 8 * 64, SW_64B);
         mma_ss<KIND_TF32>(tbase, ah, bhd, kSgIdesc, (kc > 0 || ks > 0) ? 1u : 0u);
         mma_ss<KIND_TF32>(tbase, ah, bld, kSgIdesc, 1u);
         mma_ss<KIND_TF32>(tbase, al, bhd, kSgIdesc, 1u);
@@ -156,9 +157,11 @@ __global__ void __launch_bounds__(128, 2) score_gemm_kernel(const __grid_constan
   } else {
     tc_fence_after();
     // warp w holds tile rows 32w .. 32w+31 (TMEM lanes of its quarter); each
-    // 32 x 32 block goes through a padded shared tile and out row by row, one
-    // 128-byte segment per store
-    float* tile = reinterpret_cast<float*>(lo) + warp * 32 * 33;
+    // 32 x 32 block goes through a padded shared tile (in the two chunk
+    // buffers, idle once the last MMA is done) and out row by row, one 128-byte
+    // segment per store
+    static_assert(4 * 32 * 33 * 4 <= 2 * kSgRaw, "epilogue tiles exceed the chunk buffers");
+    float* tile = reinterpret_cast<float*>(raw) + warp * 32 * 33;
 #pragma unroll 1
     for (int cc = 0; cc < kSgN; cc += 32) {
       uint32_t v[32];
