@@ -108,3 +108,36 @@ def test_plan_parity_720p_keep_sweep(keep, smooth):
     plan = lx.lx_sparse_attn_plan(Q, K, keep)
     assert lx.lx_last_device_status() == 0
     check_plan(plan.idx, plan.mask, Q.cpu(), K.cpu(), keep)
+
+
+@pytest.mark.parametrize("keep", [0.1, 0.5])
+def test_plan_large_tie_groups_take_lowest_ids(keep):
+    # key blocks cycle through three patterns, so every score row holds only
+    # three distinct values with ~100 members each: the bucket holding the k-th
+    # score has far more members than the candidate buffer, and the exact
+    # whole-row ranking must keep the lowest ids of the tied group.  Identical
+    # key blocks give bit-identical means and scores on both sides, and the
+    # three levels are far apart, so the ids must match the oracle exactly.
+    nB, d = 300, 128
+    Q, _, _ = _inputs(1, 2, 64 * nB, d, seed=11)
+    g = torch.Generator(device=DEV).manual_seed(12)
+    base = torch.randn(3, 2, 64, d, generator=g, device=DEV).to(torch.bfloat16)
+    K = torch.stack([base[j % 3] for j in range(nB)], dim=1).reshape(2, nB * 64, d).unsqueeze(0)
+    plan = lx.lx_sparse_attn_plan(Q, K, keep)
+    assert lx.lx_last_device_status() == 0
+    ref = oracle.plan_ref(Q.cpu(), K.cpu(), keep)
+    assert np.array_equal(to_np(plan.idx), ref["idx"])
+    check_plan(plan.idx, plan.mask, Q.cpu(), K.cpu(), keep)
+
+
+def test_plan_narrow_score_range_with_large_offset():
+    # all means near one common vector: the scores share a large offset and
+    # differ by a small fraction of it
+    B, H, L, d = 1, 2, 64 * 200, 128
+    g = torch.Generator(device=DEV).manual_seed(13)
+    Q = (1.0 + 0.1 * torch.randn(B, H, L, d, generator=g, device=DEV)).to(torch.bfloat16)
+    K = (1.0 + 0.1 * torch.randn(B, H, L, d, generator=g, device=DEV)).to(torch.bfloat16)
+    for keep in (0.1, 0.3):
+        plan = lx.lx_sparse_attn_plan(Q, K, keep)
+        assert lx.lx_last_device_status() == 0
+        check_plan(plan.idx, plan.mask, Q.cpu(), K.cpu(), keep)
