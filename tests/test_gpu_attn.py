@@ -124,3 +124,19 @@ def test_attn_720p_pure_noise_keep_sweep():
         assert mx <= TOL_I8_MAXABS and rl1 <= TOL_I8_RELL1, (keep, mx, rl1)
         mx, _ = compare_rows(Ob, Rb, w.L, blocks)
         assert mx <= TOL_BF16_MAXABS, (keep, mx)
+
+
+@pytest.mark.parametrize("qk_scale", [4.0, 6.0, 10.0])
+def test_attn_int8fp8_large_qk_scales(qk_scale):
+    # large Q/K magnitudes: the per-block score scale crosses the bound below
+    # which the softmax folds the INT8 magic offset into its FMA constant, so
+    # both the folded and the exact exponent paths run (V stays at scale 1)
+    B, H, L, d, keep = 1, 2, 3000, 128, 0.2
+    Q, K, _ = synth.random_qkv(B, H, L, d, seed=31, scale=qk_scale, device=DEV)
+    _, _, V = synth.random_qkv(B, H, L, d, seed=32, device=DEV)
+    plan, ref = plan_from_oracle(Q.cpu(), K.cpu(), keep, DEV)
+    O = lx.lx_sparse_attn_fwd(Q, K, V, plan, "int8fp8")
+    assert lx.lx_last_device_status() == 0
+    R = oracle.attn_ref_int8fp8(Q.cpu(), K.cpu(), V.cpu(), ref["idx"])
+    mx, rl1 = compare_rows(O, R, L, _all_blocks(B, H, L))
+    assert mx <= TOL_I8_MAXABS and rl1 <= TOL_I8_RELL1, (mx, rl1)
