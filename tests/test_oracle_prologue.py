@@ -1,0 +1,140 @@
+"""Pins of the prologue oracle (per-head RMSNorm, 3D RoPE, bf16 rounding)
+against closed forms, invariants and torch's own cast; CPU only."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+
+
+def _rand(shape, seed, scale=1.0):
+    return np.random.default_rng(seed).standard_normal(shape) * scale
+
+
+def test_rmsnorm_hand_example():
+    # one head, d = 2, x = (3, 4): mean of squares 12.5
+    x = np.array([[[[3.0, 4.0]]]])
+    w = np.array([[2.0, 0.5]])
+    y = oracle.qk_rmsnorm_ref(x, w, eps=0.0)
+    r = math.sqrt(12.5)
+    assert np.allclose(y[0, 0, 0], [2.0 * 3.0 / r, 0.5 * 4.0 / r], rtol=0, atol=1e-15)
+
+
+def test_rmsnorm_unit_rms_and_scale_invariance():
+    x = _rand((2, 3, 50, 64), 1)
+    w = np.ones((3, 64))
+    y = oracle.qk_rmsnorm_ref(x, w, eps=0.0)
+    assert np.allclose(np.sqrt(np.mean(y * y, axis=-1)), 1.0, atol=1e-13)
+    y2 = oracle.qk_rmsnorm_ref(7.5 * x, w, eps=0.0)
+    assert np.allclose(y, y2, atol=1e-13)
+    # eps damps small rows: a zero row stays zero, a tiny row is not blown up to unit RMS
+    z = np.zeros((1, 1, 1, 64))
+    assert np.all(oracle.qk_rmsnorm_ref(z, np.ones((1, 64)), eps=1e-6) == 0)
+    t = np.full((1, 1, 1, 64), 1e-6)
+    assert np.sqrt(np.mean(oracle.qk_rmsnorm_ref(t, np.ones((1, 64)), eps=1e-6) ** 2)) < 2e-3
+
+
+def test_rmsnorm_weights_per_head():
+    x = _rand((1, 2, 4, 8), 2)
+    w = np.stack([np.arange(1, 9, dtype=float), np.full(8, -1.0)])
+    y = oracle.qk_rmsnorm_ref(x, w, eps=1e-6)
+    base = oracle.qk_rmsnorm_ref(x, np.ones((2, 8)), eps=1e-6)
+    assert np.allclose(y[:, 0], base[:, 0] * w[0], atol=1e-14)
+    assert np.allclose(y[:, 1], -base[:, 1], atol=1e-14)
+
+
+def test_split_and_positions():
+    assert oracle.rope3d_split(128) == (44, 42, 42)
+    assert oracle.rope3d_split(64) == (24, 20, 20)
+    grid = (3, 4, 5)
+    pos = oracle.token_positions(60, grid)
+    n = 0
+    for t in range(3):
+        for h in range(4):
+            for w in range(5):
+                assert tuple(pos[n]) == (t, h, w)
+                n += 1
+    with pytest.raises(ValueError):
+        oracle.token_positions(61, grid)
+
+
+def test_rope_closed_form_one_pair_per_part():
+    # d = 6 splits into three parts of one pair each, frequency theta^0 = 1, so
+    # each pair turns by its own coordinate in radians
+    grid = (2, 3, 4)
+    L = 24
+    x = _rand((1, 1, L, 6), 3)
+    y = oracle.rope3d_ref(x, grid)
+    for n in range(L):
+        t, h, w = n // 12, (n // 4) % 3, n % 4
+        for part, p in enumerate((t, h, w)):
+            a, b = x[0, 0, n, 2 * part], x[0, 0, n, 2 * part + 1]
+            want = (a * math.cos(p) - b * math.sin(p), a * math.sin(p) + b * math.cos(p))
+            assert abs(y[0, 0, n, 2 * part] - want[0]) < 1e-14
+            assert abs(y[0, 0, n, 2 * part + 1] - want[1]) < 1e-14
+
+
+def test_rope_second_frequency():
+    # a part of 4 channels: pair 0 turns by p, pair 1 by p * theta^(-1/2)
+    x = np.zeros((1, 1, 8, 12))
+    x[..., 2] = 1.0          # pair 1 of the time part (channels 2, 3), d_t = 12 - 8 = 4
+    y = oracle.rope3d_ref(x, (8, 1, 1), split=(4, 4, 4))
+    for t in range(8):
+        ang = t * 10000.0 ** (-0.5)
+        assert abs(y[0, 0, t, 2] - math.cos(ang)) < 1e-14 and abs(y[0, 0, t, 3] - math.sin(ang)) < 1e-14
+
+
+def test_rope_identity_at_origin_and_norm_preserved():
+    grid = (4, 6, 8)
+    x = _rand((2, 2, 192, 128), 4)
+    y = oracle.rope3d_ref(x, grid)
+    assert np.allclose(y[:, :, 0], x[:, :, 0], atol=0)   # token 0 sits at (0, 0, 0)
+    pair_x = x[..., 0::2] ** 2 + x[..., 1::2] ** 2
+    pair_y = y[..., 0::2] ** 2 + y[..., 1::2] ** 2
+    assert np.allclose(pair_x, pair_y, rtol=1e-12)
+
+
+def test_rope_relative_position():
+    # q . k after RoPE depends only on the position difference along each axis:
+    # shifting both tokens by the same step along one axis keeps the product
+    grid = (5, 5, 5)
+    rng = np.random.default_rng(5)
+    q, k = rng.standard_normal(128), rng.standard_normal(128)
+
+    def dot(nq, nk):
+        x = np.zeros((1, 1, 125, 128))
+        x[0, 0, nq] += q
+        y1 = oracle.rope3d_ref(x, grid)[0, 0, nq]
+        x = np.zeros((1, 1, 125, 128))
+        x[0, 0, nk] += k
+        y2 = oracle.rope3d_ref(x, grid)[0, 0, nk]
+        return float(y1 @ y2)
+
+    idx = lambda t, h, w: t * 25 + h * 5 + w
+    base = dot(idx(1, 2, 0), idx(0, 1, 3))
+    assert abs(dot(idx(2, 2, 0), idx(1, 1, 3)) - base) < 1e-10      # t shifted
+    assert abs(dot(idx(1, 4, 0), idx(0, 3, 3)) - base) < 1e-10      # h shifted
+    assert abs(dot(idx(1, 2, 1), idx(0, 1, 4)) - base) < 1e-10      # w shifted
+    assert abs(dot(idx(1, 2, 0), idx(0, 2, 3)) - base) > 1e-6       # a different offset
+
+
+def test_bf16_round_matches_torch_cast():
+    # fp32 values: torch's fp32 -> bf16 cast is round to nearest even
+    x = (np.random.default_rng(6).standard_normal(200000) * np.exp(np.random.default_rng(7).uniform(-20, 20, 200000)))
+    x = x.astype(np.float32)
+    x[:4] = [0.0, 1.0 + 2 ** -8, 1.0 + 3 * 2 ** -8, -(1.0 + 2 ** -8)]   # exact ties
+    want = torch.from_numpy(x).to(torch.bfloat16).to(torch.float64).numpy()
+    got = oracle.bf16_round(x.astype(np.float64))
+    assert np.array_equal(got, want)
+
+
+def test_prologue_composition_shapes():
+    x = _rand((1, 2, 200, 64), 8, scale=3.0)
+    w = 1.0 + 0.1 * _rand((2, 64), 9)
+    r = oracle.prologue_ref(x, w, 1e-6, (2, 10, 10))
+    assert r["Y"].shape == (1, 2, 200, 64) and r["means"].shape == (1, 2, 4, 64)
+    assert r["codes"].dtype == np.int8 and r["scales"].shape == (1, 2, 4)
+    # Y is bf16-representable
+    assert np.array_equal(oracle.bf16_round(r["Y"]), r["Y"])
