@@ -124,6 +124,44 @@ lx_status lx_quantize_qk(const lx_bhld* Q, const lx_bhld* K, int8_t* qc, float* 
 lx_status lx_pool_quantize_qk(const lx_bhld* Q, const lx_bhld* K, float* mq, float* mk, int8_t* qc, float* qs,
                               int8_t* kc, float* ks, cudaStream_t stream);
 
+/* Step f1 -- the fused Q/K prologue ("600倍加速…", §高效推理算子, last
+ * paragraph: 3D RoPE and RMSNorm as fused kernels, fewer round trips through
+ * memory).  The pages give no formula; this library's reading, per tensor:
+ *   y = rope(x / sqrt(mean_c x_c^2 + eps) * w[h, c])
+ * (RMSNorm over each head's D channels, weights fp32 [H, D]), where the
+ * token at raster index n of the (T, Hh, W) grid (W fastest) has position
+ * (t, h, w) = (n / (Hh W), (n / W) mod Hh, n mod W); the head dimension is cut
+ * into the t, h and w parts of dt, dh and dw channels (even, in that order,
+ * summing to D; the default reading is D - 4 floor(D/6), 2 floor(D/6),
+ * 2 floor(D/6)), and pair i of a part of m channels turns by
+ * pos * theta^(-2i/m): (a, b) -> (a cos - b sin, a sin + b cos).
+ * The prologue's output is bf16(y); the block means and INT8 codes/scales are
+ * those of that bf16 tensor, bit-identical to lx_pool_quantize_qk run on it. */
+typedef struct lx_rope3d {
+  int64_t T, Hh, W;   /* token grid; T*Hh*W >= L */
+  int32_t dt, dh, dw; /* channels of the t, h and w parts */
+  double theta;       /* base, > 0 (10000 in the default reading) */
+} lx_rope3d;
+
+/* Bytes of the (cos, sin) table of lx_rope3d_table: 8 * (T dt + Hh dh + W dw) / 2. */
+lx_status lx_rope3d_table_size(const lx_rope3d* rope, int64_t D, size_t* bytes);
+
+/* Fills `table` (device, 16-byte aligned) with fp32 (cos, sin) pairs, the
+ * angles and their sine and cosine taken in fp64: the t part (T positions x
+ * dt/2 pairs), then the h part, then the w part.  It depends on the grid and
+ * D only, so one table serves every call of that shape. */
+lx_status lx_rope3d_table(const lx_rope3d* rope, int64_t D, float* table, cudaStream_t stream);
+
+/* The prologue of Q and K in one read of each.  wq, wk: fp32 [H, D]; table:
+ * from lx_rope3d_table; eps >= 0.  Yq, Yk: bf16 outputs (both or neither may
+ * be NULL), same shape as Q.  mq, mk: block means fp32 [B,H,nB,D] (required).
+ * qc, qs, kc, ks: INT8 codes and scales as for lx_quantize_qk (all four or
+ * none may be NULL).  L must not exceed T*Hh*W.  All pointers 16-byte
+ * aligned. */
+lx_status lx_qk_prologue(const lx_bhld* Q, const lx_bhld* K, const float* wq, const float* wk, float eps,
+                         const lx_rope3d* rope, const float* table, const lx_bhld* Yq, const lx_bhld* Yk, float* mq,
+                         float* mk, int8_t* qc, float* qs, int8_t* kc, float* ks, cudaStream_t stream);
+
 /* Step a3 -- FP8 E4M3 V ("600倍加速…", §高效推理算子: "V FP8").
  * vc: uint8 [B,H,L,D] contiguous E4M3 codes; vs: fp32 [B,H,D] scales =
  * absmax over all L tokens / 448 (1 for an all-zero channel);

@@ -28,7 +28,6 @@ Pins for every function live in ``tests/test_oracle_prologue.py``.
 """
 from __future__ import annotations
 
-import math
 
 import numpy as np
 

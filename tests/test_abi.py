@@ -133,3 +133,29 @@ def test_fwd_plan_and_workspace_checks(lib):
     assert lib.lx_sparse_attn_fwd(ctypes.byref(q), ctypes.byref(q), ctypes.byref(q), ctypes.byref(good), 7,
                                   ctypes.byref(q), 0x100000, 1 << 30, s) == _abi.LX_ERR_INVALID
     assert lib.lx_debug_wait_timeout(0, s) == _abi.LX_ERR_INVALID
+
+
+def test_prologue_argument_errors_before_launch(lib):
+    s = ctypes.c_void_p(0)
+    q = _view(L=1000)
+    good = _abi.LxRope3d(4, 16, 16, 44, 42, 42, 10000.0)
+    n = ctypes.c_size_t()
+    assert lib.lx_rope3d_table_size(ctypes.byref(good), 128, ctypes.byref(n)) == 0
+    assert n.value == 8 * (4 * 22 + 16 * 21 + 16 * 21)
+    for bad in (_abi.LxRope3d(4, 16, 16, 43, 43, 42, 10000.0),     # odd parts
+                _abi.LxRope3d(4, 16, 16, 44, 42, 40, 10000.0),     # parts do not add up to D
+                _abi.LxRope3d(4, 16, 16, 44, 42, 42, 0.0),         # theta
+                _abi.LxRope3d(0, 16, 16, 44, 42, 42, 10000.0)):    # empty grid
+        assert lib.lx_rope3d_table_size(ctypes.byref(bad), 128, ctypes.byref(n)) == _abi.LX_ERR_INVALID
+    assert lib.lx_rope3d_table(ctypes.byref(good), 128, 0x20008, s) == _abi.LX_ERR_ALIGN
+    p = [0x20000, 0x30000, 0x40000, 0x50000, 0x60000, 0x70000]   # mq mk qc qs kc ks
+    call = lambda rope=good, yq=None, yk=None, outs=p, eps=1e-6, X=q: lib.lx_qk_prologue(
+        ctypes.byref(X), ctypes.byref(X), 0x80000, 0x90000, eps, ctypes.byref(rope), 0xA0000,
+        ctypes.byref(yq) if yq is not None else None, ctypes.byref(yk) if yk is not None else None, *outs, s)
+    small = _abi.LxRope3d(3, 16, 16, 44, 42, 42, 10000.0)         # 768 positions < L = 1000
+    assert call(rope=small) == _abi.LX_ERR_INVALID
+    assert call(eps=-1.0) == _abi.LX_ERR_INVALID
+    assert call(yq=q) == _abi.LX_ERR_INVALID                        # one output without the other
+    assert call(outs=[0x20000, 0x30000, 0x40000, None, 0x60000, 0x70000]) == _abi.LX_ERR_INVALID
+    assert call(outs=[None, 0x30000, 0x40000, 0x50000, 0x60000, 0x70000]) == _abi.LX_ERR_INVALID
+    assert call(outs=[0x20008, 0x30000, 0x40000, 0x50000, 0x60000, 0x70000]) == _abi.LX_ERR_ALIGN

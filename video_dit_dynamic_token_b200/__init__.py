@@ -167,6 +167,61 @@ def lx_pool_quantize_qk(Q, K, out=None, stream=None):
     return out
 
 
+def rope3d_default_split(D):
+    """The default (t, h, w) channel split of a head dimension D."""
+    q = D // 6
+    return D - 4 * q, 2 * q, 2 * q
+
+
+def _rope(grid, D, theta, split):
+    dt, dh, dw = rope3d_default_split(D) if split is None else split
+    T, Hh, W = grid
+    return _abi.LxRope3d(T, Hh, W, dt, dh, dw, float(theta))
+
+
+def lx_rope3d_table(grid, D, theta=10000.0, split=None, device="cuda", stream=None):
+    """The (cos, sin) table of the 3D RoPE of a (T, Hh, W) grid, fp32 on the device."""
+    lib = _abi.load()
+    r = _rope(grid, D, theta, split)
+    n = ctypes.c_size_t()
+    _check(lib.lx_rope3d_table_size(ctypes.byref(r), D, ctypes.byref(n)), "lx_rope3d_table_size")
+    table = torch.empty(max(n.value // 4, 4), dtype=torch.float32, device=device)
+    _check(lib.lx_rope3d_table(ctypes.byref(r), D, _ptr(table), _stream(stream)), "lx_rope3d_table")
+    return table
+
+
+def lx_qk_prologue(Q, K, wq, wk, eps, grid, theta=10000.0, split=None, table=None, with_y=True, with_codes=True,
+                   stream=None):
+    """Per-head RMSNorm + 3D RoPE of Q and K, with the block means and INT8 codes
+    of the bf16 result, in one pass: dict(Yq, Yk, mq, mk, qc, qs, kc, ks)."""
+    lib = _abi.load()
+    B, H, L, D = Q.shape
+    nB = (L + LX_BLOCK - 1) // LX_BLOCK
+    dev = Q.device
+    if table is None:
+        table = lx_rope3d_table(grid, D, theta, split, dev, stream)
+    r = _rope(grid, D, theta, split)
+    out = {"mq": torch.empty((B, H, nB, D), dtype=torch.float32, device=dev),
+           "mk": torch.empty((B, H, nB, D), dtype=torch.float32, device=dev)}
+    yq = yk = None
+    if with_y:
+        out["Yq"] = torch.empty((B, H, L, D), dtype=torch.bfloat16, device=dev)
+        out["Yk"] = torch.empty((B, H, L, D), dtype=torch.bfloat16, device=dev)
+        yq, yk = bhld(out["Yq"]), bhld(out["Yk"])
+    if with_codes:
+        out["qc"] = torch.empty((B, H, L, D), dtype=torch.int8, device=dev)
+        out["qs"] = torch.empty((B, H, nB), dtype=torch.float32, device=dev)
+        out["kc"] = torch.empty((B, H, L, D), dtype=torch.int8, device=dev)
+        out["ks"] = torch.empty((B, H, nB), dtype=torch.float32, device=dev)
+    q, k = bhld(Q), bhld(K)
+    p = lambda name: _ptr(out[name]) if name in out else None
+    _check(lib.lx_qk_prologue(ctypes.byref(q), ctypes.byref(k), _ptr(wq), _ptr(wk), float(eps), ctypes.byref(r),
+                              _ptr(table), ctypes.byref(yq) if yq is not None else None,
+                              ctypes.byref(yk) if yk is not None else None, p("mq"), p("mk"), p("qc"), p("qs"),
+                              p("kc"), p("ks"), _stream(stream)), "lx_qk_prologue")
+    return out
+
+
 def lx_quantize_v(V, out=None, amax_ws=None, stream=None):
     lib = _abi.load()
     B, H, L, D = V.shape

@@ -34,6 +34,11 @@ class LxPlan(ctypes.Structure):
                 ("nB", _c_i64), ("k", _c_i64), ("block", ctypes.c_int32)]
 
 
+class LxRope3d(ctypes.Structure):
+    _fields_ = [("T", _c_i64), ("Hh", _c_i64), ("W", _c_i64), ("dt", ctypes.c_int32), ("dh", ctypes.c_int32),
+                ("dw", ctypes.c_int32), ("theta", _dbl)]
+
+
 _P = ctypes.POINTER
 SIGNATURES = {
     "lx_plan_size": [_c_i64, _c_i64, _c_i64, _c_i64, _dbl, _P(_c_i64), _P(_c_sz), _P(_c_sz), _P(_c_sz)],
@@ -42,6 +47,10 @@ SIGNATURES = {
     "lx_sparse_attn_plan": [_P(LxBhld), _P(LxBhld), _dbl, _P(LxPlan), _vp, _c_sz, _vp],
     "lx_quantize_qk": [_P(LxBhld), _P(LxBhld), _vp, _vp, _vp, _vp, _vp],
     "lx_pool_quantize_qk": [_P(LxBhld), _P(LxBhld), _vp, _vp, _vp, _vp, _vp, _vp, _vp],
+    "lx_rope3d_table_size": [_P(LxRope3d), _c_i64, _P(_c_sz)],
+    "lx_rope3d_table": [_P(LxRope3d), _c_i64, _vp, _vp],
+    "lx_qk_prologue": [_P(LxBhld), _P(LxBhld), _vp, _vp, ctypes.c_float, _P(LxRope3d), _vp, _P(LxBhld), _P(LxBhld),
+                       _vp, _vp, _vp, _vp, _vp, _vp, _vp],
     "lx_quantize_v": [_P(LxBhld), _vp, _vp, _vp, _vp],
     "lx_quantize_v_noalloc": [_P(LxBhld), _vp, _vp, _vp],
     "lx_attn_bf16": [_P(LxBhld), _P(LxBhld), _P(LxBhld), _P(LxPlan), _P(LxBhld), _vp],

@@ -114,16 +114,24 @@ bool make_map(CUtensorMap* m, const void* ptr, CUtensorMapDataType dt, int esz, 
 // ---------------------------------------------------------------- launchers
 template <int D>
 lx_status launch_qk_pass(const lx_bhld* Q, const lx_bhld* K, float* mq, float* mk, int8_t* qc, float* qs, int8_t* kc,
-                         float* ks, cudaStream_t s) {
+                         float* ks, cudaStream_t s, const lx::ProParams* pro = nullptr) {
   const int64_t nB = n_blocks(Q->L);
   dim3 grid((unsigned)(Q->B * Q->H * nB), 2);
   const int H = (int)Q->H, L = (int)Q->L;
-  if (mq && qc)
-    lx::qk_block_pass_kernel<D, true, true><<<grid, 128, 0, s>>>(view(Q), view(K), mq, mk, qc, kc, qs, ks, H, L, (int)nB);
-  else if (mq)
-    lx::qk_block_pass_kernel<D, true, false><<<grid, 128, 0, s>>>(view(Q), view(K), mq, mk, qc, kc, qs, ks, H, L, (int)nB);
-  else
-    lx::qk_block_pass_kernel<D, false, true><<<grid, 128, 0, s>>>(view(Q), view(K), mq, mk, qc, kc, qs, ks, H, L, (int)nB);
+  const lx::ProParams pp = pro ? *pro : lx::ProParams{};
+  const lx::BhldView vq = view(Q), vk = view(K);
+  if (pro) {
+    if (qc)
+      lx::qk_block_pass_kernel<D, true, true, true><<<grid, 128, 0, s>>>(vq, vk, mq, mk, qc, kc, qs, ks, H, L, (int)nB, pp);
+    else
+      lx::qk_block_pass_kernel<D, true, false, true><<<grid, 128, 0, s>>>(vq, vk, mq, mk, qc, kc, qs, ks, H, L, (int)nB, pp);
+  } else if (mq && qc) {
+    lx::qk_block_pass_kernel<D, true, true, false><<<grid, 128, 0, s>>>(vq, vk, mq, mk, qc, kc, qs, ks, H, L, (int)nB, pp);
+  } else if (mq) {
+    lx::qk_block_pass_kernel<D, true, false, false><<<grid, 128, 0, s>>>(vq, vk, mq, mk, qc, kc, qs, ks, H, L, (int)nB, pp);
+  } else {
+    lx::qk_block_pass_kernel<D, false, true, false><<<grid, 128, 0, s>>>(vq, vk, mq, mk, qc, kc, qs, ks, H, L, (int)nB, pp);
+  }
   return launch_status();
 }
 
@@ -345,6 +353,79 @@ lx_status lx_pool_quantize_qk(const lx_bhld* Q, const lx_bhld* K, float* mq, flo
   if (!al16(mq) || !al16(mk) || !al16(qc) || !al16(kc) || !al16(qs) || !al16(ks)) return LX_ERR_ALIGN;
   return Q->D == 128 ? launch_qk_pass<128>(Q, K, mq, mk, qc, qs, kc, ks, stream)
                      : launch_qk_pass<64>(Q, K, mq, mk, qc, qs, kc, ks, stream);
+}
+
+// ---------------------------------------------------------------- prologue (3D RoPE + RMSNorm)
+namespace {
+lx_status check_rope(const lx_rope3d* r, int64_t D) {
+  if (!r) return LX_ERR_INVALID;
+  if (D != 64 && D != 128) return LX_ERR_UNSUPPORTED;
+  if (r->T < 1 || r->Hh < 1 || r->W < 1 || r->T * r->Hh * r->W > (int64_t)1 << 30) return LX_ERR_INVALID;
+  if (r->dt < 0 || r->dh < 0 || r->dw < 0 || (r->dt | r->dh | r->dw) & 1 || r->dt + r->dh + r->dw != D)
+    return LX_ERR_INVALID;
+  if (!(r->theta > 0.0) || !std::isfinite(r->theta)) return LX_ERR_INVALID;
+  return LX_OK;
+}
+int64_t rope_entries(const lx_rope3d* r) { return r->T * (r->dt / 2) + r->Hh * (r->dh / 2) + r->W * (r->dw / 2); }
+}  // namespace
+
+lx_status lx_rope3d_table_size(const lx_rope3d* rope, int64_t D, size_t* bytes) {
+  lx_status st = check_rope(rope, D);
+  if (st != LX_OK) return st;
+  if (!bytes) return LX_ERR_INVALID;
+  *bytes = sizeof(float) * 2 * (size_t)rope_entries(rope);
+  return LX_OK;
+}
+
+lx_status lx_rope3d_table(const lx_rope3d* rope, int64_t D, float* table, cudaStream_t stream) {
+  lx_status st = check_rope(rope, D);
+  if (st != LX_OK) return st;
+  if (!table) return LX_ERR_INVALID;
+  if (!al16(table)) return LX_ERR_ALIGN;
+  const int64_t n = rope_entries(rope);
+  if (n == 0) return LX_OK;
+  const unsigned blocks = (unsigned)std::min<int64_t>((n + 255) / 256, 1024);
+  lx::rope3d_table_kernel<<<blocks, 256, 0, stream>>>(reinterpret_cast<float2*>(table), (int)rope->T, (int)rope->Hh,
+                                                       (int)rope->W, rope->dt / 2, rope->dh / 2, rope->dw / 2,
+                                                       rope->theta);
+  return launch_status();
+}
+
+lx_status lx_qk_prologue(const lx_bhld* Q, const lx_bhld* K, const float* wq, const float* wk, float eps,
+                         const lx_rope3d* rope, const float* table, const lx_bhld* Yq, const lx_bhld* Yk, float* mq,
+                         float* mk, int8_t* qc, float* qs, int8_t* kc, float* ks, cudaStream_t stream) {
+  lx_status st;
+  if ((st = check_bhld(Q)) != LX_OK || (st = check_bhld(K)) != LX_OK) return st;
+  if (!same_shape(Q, K)) return LX_ERR_INVALID;
+  if ((st = check_rope(rope, Q->D)) != LX_OK) return st;
+  if (Q->L > rope->T * rope->Hh * rope->W) return LX_ERR_INVALID;
+  if (!wq || !wk || !table || !mq || !mk || !(eps >= 0.f) || !std::isfinite(eps)) return LX_ERR_INVALID;
+  if ((qc == nullptr) != (kc == nullptr) || (qc == nullptr) != (qs == nullptr) || (qs == nullptr) != (ks == nullptr))
+    return LX_ERR_INVALID;
+  if ((Yq == nullptr) != (Yk == nullptr)) return LX_ERR_INVALID;
+  if (Yq) {
+    if ((st = check_bhld(Yq)) != LX_OK || (st = check_bhld(Yk)) != LX_OK) return st;
+    if (!same_shape(Q, Yq) || !same_shape(Q, Yk)) return LX_ERR_INVALID;
+  }
+  if (!al16(wq) || !al16(wk) || !al16(table) || !al16(mq) || !al16(mk)) return LX_ERR_ALIGN;
+  if (qc && (!al16(qc) || !al16(kc) || !al16(qs) || !al16(ks))) return LX_ERR_ALIGN;
+  lx::ProParams pro{};
+  pro.wq = wq;
+  pro.wk = wk;
+  pro.table = reinterpret_cast<const float2*>(table);
+  if (Yq) {
+    pro.yq = lx::BhldOut{reinterpret_cast<__nv_bfloat16*>(Yq->data), Yq->sB, Yq->sH, Yq->sL};
+    pro.yk = lx::BhldOut{reinterpret_cast<__nv_bfloat16*>(Yk->data), Yk->sB, Yk->sH, Yk->sL};
+  }
+  pro.eps = eps;
+  pro.Hh = (int)rope->Hh;
+  pro.W = (int)rope->W;
+  pro.dt2 = rope->dt / 2;
+  pro.dh2 = rope->dh / 2;
+  pro.offh = (int)(rope->T * (rope->dt / 2));
+  pro.offw = pro.offh + (int)(rope->Hh * (rope->dh / 2));
+  return Q->D == 128 ? launch_qk_pass<128>(Q, K, mq, mk, qc, qs, kc, ks, stream, &pro)
+                     : launch_qk_pass<64>(Q, K, mq, mk, qc, qs, kc, ks, stream, &pro);
 }
 
 lx_status lx_quantize_v(const lx_bhld* V, uint8_t* vc, float* vs, uint32_t* amax_ws, cudaStream_t stream) {

@@ -56,6 +56,31 @@ __device__ __forceinline__ uint32_t e4m3x4(float a, float b, float c, float d) {
 }
 
 // ---------------------------------------------------------------------------
+// Prologue parameters of the Q/K block pass (per-head RMSNorm and 3D RoPE,
+// "600倍加速…", §高效推理算子, last paragraph: 3D RoPE and RMSNorm as fused
+// kernels; the formulas are this library's reading):
+//   y = rope(x / sqrt(mean_c x_c^2 + eps) * w[h, c]).
+// The head dimension is split into the t, h and w parts (dt2, dh2, dw2 channel
+// pairs, in that order); pair i of a part turns by pos * theta^(-2i/m), whose
+// (cos, sin) sit in `table` at part base + pos * pairs + i.  The token at raster
+// index n of the (T, Hh, W) grid has (t, h, w) = (n / (Hh W), (n / W) mod Hh,
+// n mod W).  yq / yk receive bf16(y) when their pointer is not null.
+struct BhldOut {  // bf16 [B,H,L,D] output with element strides
+  __nv_bfloat16* p;
+  long long sB, sH, sL;
+};
+struct ProParams {
+  const float* wq;     // [H, D]
+  const float* wk;     // [H, D]
+  const float2* table; // (cos, sin) per (part, position, pair)
+  BhldOut yq, yk;
+  float eps;
+  int Hh, W;
+  int dt2, dh2;        // channel pairs of the t and h parts (the w part has D/2 - dt2 - dh2)
+  int offh, offw;      // table offsets of the h and w parts (entries)
+};
+
+// ---------------------------------------------------------------------------
 // Q/K block pass (steps a1 and a3 in one read): one 128-thread CTA per
 // (tensor, b*h, 64-token block).  The D/8 16-byte chunks of a row go to
 // consecutive lanes (a warp loads whole rows, coalesced) and the 128/(D/8) row
@@ -67,11 +92,14 @@ __device__ __forceinline__ uint32_t e4m3x4(float a, float b, float c, float d) {
 // becomes rint(x * inv) clamped to +-127; the scale a/127 (1 for an all-zero
 // block) is stored per block.  Either part may be switched off, so the pool,
 // the quantiser and the fused pass share one code path and agree bit for bit.
-template <int D, bool MEANS, bool CODES>
+// PRO: each valid row is first replaced by the bf16 prologue output (above),
+// so the means and codes are those of that bf16 tensor.
+template <int D, bool MEANS, bool CODES, bool PRO>
 __global__ void __launch_bounds__(128) qk_block_pass_kernel(BhldView q, BhldView k, float* __restrict__ mq,
                                                            float* __restrict__ mk, int8_t* __restrict__ qc,
                                                            int8_t* __restrict__ kc, float* __restrict__ qs,
-                                                           float* __restrict__ ks, int H, int L, int nB) {
+                                                           float* __restrict__ ks, int H, int L, int nB,
+                                                           ProParams pro) {
   constexpr int CH = D / 8;      // 16-byte chunks per row
   constexpr int RG = 128 / CH;   // row groups in the CTA
   constexpr int NR = kBlock / RG;  // rows per thread (= D/16)
@@ -88,6 +116,67 @@ __global__ void __launch_bounds__(128) qk_block_pass_kernel(BhldView q, BhldView
   uint4 v[NR];
 #pragma unroll
   for (int i = 0; i < NR; ++i) v[i] = r + RG * i < cnt ? ld_stream_v4(src + (long long)(RG * i) * X.sL) : make_uint4(0, 0, 0, 0);
+  if constexpr (PRO) {
+    const bool isk = blockIdx.y != 0;
+    // this thread's 8 channels: weights and, for each of its 4 pairs, the
+    // table part (0 t, 1 h, 2 w), base and pairs per position
+    const float4* wrow = reinterpret_cast<const float4*>((isk ? pro.wk : pro.wq) + h * D + c * 8);
+    const float4 w0 = __ldg(wrow), w1 = __ldg(wrow + 1);
+    const float wv[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+    int pax[4], pbase[4], pstride[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int pi = 4 * c + j;
+      if (pi < pro.dt2) {
+        pax[j] = 0; pbase[j] = pi; pstride[j] = pro.dt2;
+      } else if (pi < pro.dt2 + pro.dh2) {
+        pax[j] = 1; pbase[j] = pro.offh + (pi - pro.dt2); pstride[j] = pro.dh2;
+      } else {
+        pax[j] = 2; pbase[j] = pro.offw + (pi - pro.dt2 - pro.dh2); pstride[j] = D / 2 - pro.dt2 - pro.dh2;
+      }
+    }
+    const BhldOut Y = isk ? pro.yk : pro.yq;
+#pragma unroll
+    for (int i = 0; i < NR; ++i) {
+      const int row = r + RG * i;
+      const uint32_t wd[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
+      float x[8];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        x[2 * e] = bf16lo(wd[e]);
+        x[2 * e + 1] = bf16hi(wd[e]);
+      }
+      float ss = 0.f;
+#pragma unroll
+      for (int e = 0; e < 8; ++e) ss = fmaf(x[e], x[e], ss);
+      // the row's D/8 chunks sit in consecutive lanes: fold them (every lane
+      // takes part, rows past L included, whose values are zero)
+#pragma unroll
+      for (int off = 1; off < CH; off <<= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
+      if (row < cnt) {
+        const float inv = 1.0f / sqrtf(ss / (float)D + pro.eps);
+        const int n = t0 + row;
+        const int nw = n / pro.W;
+        const int pw = n - nw * pro.W;
+        const int pt = nw / pro.Hh;
+        const int ph = nw - pt * pro.Hh;
+        uint32_t o[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const int pos = pax[j] == 0 ? pt : (pax[j] == 1 ? ph : pw);
+          const float2 cs = __ldg(pro.table + pbase[j] + pos * pstride[j]);
+          const float xa = (x[2 * j] * inv) * wv[2 * j];
+          const float xb = (x[2 * j + 1] * inv) * wv[2 * j + 1];
+          const float y0 = fmaf(xa, cs.x, -xb * cs.y);
+          const float y1 = fmaf(xa, cs.y, xb * cs.x);
+          __nv_bfloat162 yb = __floats2bfloat162_rn(y0, y1);
+          o[j] = *reinterpret_cast<uint32_t*>(&yb);
+        }
+        v[i] = make_uint4(o[0], o[1], o[2], o[3]);
+        if (Y.p) *reinterpret_cast<uint4*>(Y.p + b * Y.sB + h * Y.sH + (long long)n * Y.sL + c * 8) = v[i];
+      }
+    }
+  }
   __shared__ float part[MEANS ? 4 : 1][MEANS ? D : 1];
   __shared__ float red[4];
   if constexpr (MEANS) {
@@ -254,6 +343,30 @@ __global__ void __launch_bounds__(128, 4) v_quant_kernel(BhldView v, const uint3
     for (int i = 0; i < NR; ++i) x[i] = xn[i];
     bh = bhn;
     blk = blkn;
+  }
+}
+
+// ---------------------------------------------------------------------------
+// 3D RoPE table: entry e of the t part (then the h part, then the w part) is
+// (cos, sin) of pos * theta^(-2i/m) for position pos and pair i of a part of m
+// channels; the angle and its sine and cosine are taken in fp64 and rounded
+// to fp32 once.
+__global__ void rope3d_table_kernel(float2* __restrict__ table, int T, int Hh, int W, int dt2, int dh2, int dw2,
+                                    double theta) {
+  const int nt = T * dt2, nh = Hh * dh2, nw = W * dw2;
+  for (int e = blockIdx.x * blockDim.x + threadIdx.x; e < nt + nh + nw; e += gridDim.x * blockDim.x) {
+    int pos, i, pairs;
+    if (e < nt) {
+      pos = e / dt2; i = e - pos * dt2; pairs = dt2;
+    } else if (e < nt + nh) {
+      pos = (e - nt) / dh2; i = (e - nt) - pos * dh2; pairs = dh2;
+    } else {
+      pos = (e - nt - nh) / dw2; i = (e - nt - nh) - pos * dw2; pairs = dw2;
+    }
+    const double ang = (double)pos * pow(theta, -(double)i / (double)pairs);  // -2i/m with m = 2 pairs
+    double sn, cs;
+    sincos(ang, &sn, &cs);
+    table[e] = make_float2((float)cs, (float)sn);
   }
 }
 
