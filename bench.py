@@ -159,9 +159,20 @@ def run_ours(args, rank, world, local_rank):
         # Q/K block pass (means + INT8 codes), score GEMM, top-k, V absmax, V codes, attention
         launches_per_step = 6
         names = ["pool_quant_qk", "score_topk", "quant_v", "attn"]
+        if args.prologue:
+            names[0] = "qk_prologue"
     else:
         launches_per_step = 4  # pool, score GEMM, top-k, attention
         names = ["pool", "score_topk", "attn"]
+
+    # --prologue: the Q/K pass also applies per-head RMSNorm and the 3D RoPE of
+    # the workload's grid (random per-head weights; the table is built once)
+    pro = None
+    if args.prologue and mode == "int8fp8":
+        g = torch.Generator(device="cpu").manual_seed(1234 + rank)
+        wq = (1.0 + 0.2 * torch.randn(H, d, generator=g)).float().to(dev)
+        wk = (1.0 + 0.2 * torch.randn(H, d, generator=g)).float().to(dev)
+        pro = dict(wq=wq, wk=wk, table=lx.lx_rope3d_table(w.grid, d, device=dev))
 
     def step(ev=None):
         marks = iter(range(len(names) + 1))
@@ -170,7 +181,9 @@ def run_ours(args, rank, world, local_rank):
             if ev is not None:
                 ev[i].record(stream)
         mark()
-        if mode == "int8fp8":
+        if pro is not None:
+            lx.lx_qk_prologue_into(Q, K, pro["wq"], pro["wk"], 1e-6, w.grid, pro["table"], mq, mk, qc, qs, kc, ks)
+        elif mode == "int8fp8":
             lx.lx_pool_quantize_qk(Q, K, out=(mq, mk, qc, qs, kc, ks))
         else:
             lx.lx_pool_means(Q, K, out=(mq, mk))
@@ -261,7 +274,7 @@ def run_ours(args, rank, world, local_rank):
     plan_out_b = B * H * nB * k * 4 + B * H * nB * ((nB + 31) // 32) * 4
     phase_bytes = {"score_topk": means_b + plan_out_b}
     if mode == "int8fp8":
-        phase_bytes["pool_quant_qk"] = 2 * N * 2 + 2 * N + means_b + 2 * B * H * nB * 4
+        phase_bytes[names[0]] = 2 * N * 2 + 2 * N + means_b + 2 * B * H * nB * 4
         phase_bytes["quant_v"] = 2 * N * 2 + N + B * H * d * 4  # V read twice: the channel scale needs all of V
     else:
         phase_bytes["pool"] = 2 * N * 2 + means_b
@@ -377,6 +390,8 @@ def main():
                     help="grid shape (the headline is 720p; the others are characterisation runs)")
     ap.add_argument("--mode", default=MODE, choices=["int8fp8", "bf16"])
     ap.add_argument("--keep", type=float, default=0.0, help="override the workload's keep ratio (sweeps)")
+    ap.add_argument("--prologue", action="store_true",
+                    help="int8fp8: the Q/K pass also applies per-head RMSNorm and 3D RoPE (lx_qk_prologue)")
     args = ap.parse_args()
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))

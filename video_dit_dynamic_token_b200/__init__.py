@@ -222,6 +222,22 @@ def lx_qk_prologue(Q, K, wq, wk, eps, grid, theta=10000.0, split=None, table=Non
     return out
 
 
+def lx_qk_prologue_into(Q, K, wq, wk, eps, grid, table, mq, mk, qc=None, qs=None, kc=None, ks=None, Yq=None, Yk=None,
+                        theta=10000.0, split=None, stream=None):
+    """lx_qk_prologue into caller buffers (no allocation): means, optional codes
+    and optional bf16 outputs."""
+    lib = _abi.load()
+    D = Q.shape[-1]
+    r = _rope(grid, D, theta, split)
+    q, k = bhld(Q), bhld(K)
+    yq = bhld(Yq) if Yq is not None else None
+    yk = bhld(Yk) if Yk is not None else None
+    _check(lib.lx_qk_prologue(ctypes.byref(q), ctypes.byref(k), _ptr(wq), _ptr(wk), float(eps), ctypes.byref(r),
+                              _ptr(table), ctypes.byref(yq) if yq is not None else None,
+                              ctypes.byref(yk) if yk is not None else None, _ptr(mq), _ptr(mk), _ptr(qc), _ptr(qs),
+                              _ptr(kc), _ptr(ks), _stream(stream)), "lx_qk_prologue")
+
+
 def lx_quantize_v(V, out=None, amax_ws=None, stream=None):
     lib = _abi.load()
     B, H, L, D = V.shape

@@ -136,8 +136,28 @@ __global__ void __launch_bounds__(128) qk_block_pass_kernel(BhldView q, BhldView
       }
     }
     const BhldOut Y = isk ? pro.yk : pro.yq;
+    // grid position of this thread's first row; the later rows (RG apart) are
+    // reached by adding to w and carrying into h and t
+    int pt, ph, pw;
+    {
+      const int n = t0 + r;
+      const int nw = n / pro.W;
+      pw = n - nw * pro.W;
+      pt = nw / pro.Hh;
+      ph = nw - pt * pro.Hh;
+    }
 #pragma unroll
     for (int i = 0; i < NR; ++i) {
+      if (i > 0) {
+        pw += RG;
+        while (pw >= pro.W) {
+          pw -= pro.W;
+          if (++ph == pro.Hh) {
+            ph = 0;
+            ++pt;
+          }
+        }
+      }
       const int row = r + RG * i;
       const uint32_t wd[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
       float x[8];
@@ -154,12 +174,8 @@ __global__ void __launch_bounds__(128) qk_block_pass_kernel(BhldView q, BhldView
 #pragma unroll
       for (int off = 1; off < CH; off <<= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
       if (row < cnt) {
-        const float inv = 1.0f / sqrtf(ss / (float)D + pro.eps);
+        const float inv = rsqrtf(ss * (1.0f / (float)D) + pro.eps);  // within 2 fp32 ulps
         const int n = t0 + row;
-        const int nw = n / pro.W;
-        const int pw = n - nw * pro.W;
-        const int pt = nw / pro.Hh;
-        const int ph = nw - pt * pro.Hh;
         uint32_t o[4];
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
