@@ -9,5 +9,5 @@ from .sparse_attn_ref import (BLOCK, E4M3_MAX, attn_int8fp8_from_codes, attn_ref
                               e4m3_encode, e4m3_round, keep_count, kth_threshold, max_abs_err,
                               n_blocks, plan_mask, plan_ref, quant_qk_ref, quant_v_ref,
                               rel_l1_err, select_topk)
-from .prologue_ref import (ROPE_THETA, bf16_round, prologue_ref, qk_rmsnorm_ref, rope3d_ref,  # noqa: F401
-                           rope3d_split, token_positions)
+from .prologue_ref import (ROPE_THETA, bf16_round, k_channel_mean_ref, prologue_ref,  # noqa: F401
+                           qk_rmsnorm_ref, quant_k_smooth_ref, rope3d_ref, rope3d_split, token_positions)

@@ -1,5 +1,6 @@
 """CPU oracle for the fused Q/K prologue: per-head RMSNorm, 3D RoPE, then the
-block means and INT8 codes of the result (plain numpy, fp64).
+block means and INT8 codes of the result; and for the K-smoothing variant of
+the INT8 quantiser (plain numpy, fp64).
 
 TEST INFRASTRUCTURE ONLY, like ``sparse_attn_ref``: only ``tests/`` use it; it
 shares no code with the CUDA library.
@@ -99,3 +100,24 @@ def prologue_ref(X, w, eps: float, grid, theta: float = ROPE_THETA, split=None) 
     Y = bf16_round(rope3d_ref(qk_rmsnorm_ref(X, w, eps), grid, theta, split))
     codes, scales = quant_qk_ref(Y)
     return {"Y": Y, "means": block_means(Y), "codes": codes, "scales": scales}
+
+
+# --------------------------------------------------------------------------
+# K smoothing (a variant: not on the pages)
+# --------------------------------------------------------------------------
+# Subtracting one vector m from every key changes each score row by the constant
+# q.m, which the softmax removes, so the attention is unchanged; quantising
+# K - m instead of K shrinks the INT8 error when K has large channel offsets.
+# This library's reading: m = the per-(b, h, channel) mean of K over all L
+# tokens, taken in fp64 and rounded to fp32 once; the codes are those of
+# fl32(K - m) by the INT8 rule of ``quant_qk_ref``.
+
+def k_channel_mean_ref(K) -> np.ndarray:
+    """fp32 [B,H,D]: fl32(mean over tokens of K), the mean taken in fp64."""
+    return _f64(K).mean(axis=2).astype(np.float32)
+
+
+def quant_k_smooth_ref(K, km) -> tuple:
+    """INT8 codes and scales of fl32(K - km) (km fp32 [B,H,D])."""
+    x = (_f64(K).astype(np.float32) - np.asarray(km, dtype=np.float32)[:, :, None, :]).astype(np.float32)
+    return quant_qk_ref(x)

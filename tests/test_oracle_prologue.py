@@ -138,3 +138,64 @@ def test_prologue_composition_shapes():
     assert r["codes"].dtype == np.int8 and r["scales"].shape == (1, 2, 4)
     # Y is bf16-representable
     assert np.array_equal(oracle.bf16_round(r["Y"]), r["Y"])
+
+
+def test_k_channel_mean_and_zero_mean_after_shift():
+    K = torch.from_numpy(_rand((1, 2, 300, 64), 10, scale=2.0) + 5.0).to(torch.bfloat16)
+    km = oracle.k_channel_mean_ref(K)
+    want = K.double().mean(dim=2).float().numpy()
+    assert np.array_equal(km, want)
+    Kd = K.double().numpy()
+    assert np.abs((Kd - km[:, :, None, :].astype(np.float64)).mean(axis=2)).max() < 1e-6
+    c = torch.full((1, 1, 70, 64), 1.25, dtype=torch.bfloat16)
+    assert np.all(oracle.k_channel_mean_ref(c) == np.float32(1.25))
+
+
+def test_smoothing_leaves_exact_attention_unchanged():
+    # softmax over keys removes the per-row constant q.m
+    rng = np.random.default_rng(11)
+    B, H, L, d = 1, 2, 200, 64
+    Q = torch.from_numpy(rng.standard_normal((B, H, L, d))).to(torch.bfloat16)
+    K = torch.from_numpy(rng.standard_normal((B, H, L, d)) + rng.standard_normal((1, H, 1, d)) * 4).to(torch.bfloat16)
+    V = torch.from_numpy(rng.standard_normal((B, H, L, d))).to(torch.bfloat16)
+    idx = oracle.plan_ref(Q, K, 0.5)["idx"]
+    km = oracle.k_channel_mean_ref(K).astype(np.float64)
+    Ks = K.double().numpy() - km[:, :, None, :]
+    O1 = oracle.attn_ref_exact(Q, K, V, idx)
+    O2 = oracle.attn_ref_exact(Q, Ks, V, idx)
+    assert np.abs(O1 - O2).max() < 1e-12
+
+
+def test_smoothing_reduces_int8_error_on_offset_keys():
+    # keys with a large common channel offset: the INT8 error of the smoothed
+    # codes against the exact attention is much smaller
+    rng = np.random.default_rng(12)
+    B, H, L, d = 1, 1, 512, 64
+    Q = torch.from_numpy(rng.standard_normal((B, H, L, d))).to(torch.bfloat16)
+    off = rng.standard_normal((1, 1, 1, d)) * 8
+    K = torch.from_numpy(rng.standard_normal((B, H, L, d)) + off).to(torch.bfloat16)
+    V = torch.from_numpy(rng.standard_normal((B, H, L, d))).to(torch.bfloat16)
+    idx = oracle.plan_ref(Q, K, 0.5)["idx"]
+    R = oracle.attn_ref_exact(Q, K, V, idx)
+    qc, sq = oracle.quant_qk_ref(Q)
+    vc, sv = oracle.quant_v_ref(V)
+    kc, sk = oracle.quant_qk_ref(K)
+    ks_c, ks_s = oracle.quant_k_smooth_ref(K, oracle.k_channel_mean_ref(K))
+    e_plain = oracle.rel_l1_err(oracle.attn_int8fp8_from_codes(qc, sq, kc, sk, vc, sv, idx, L), R)
+    e_smooth = oracle.rel_l1_err(oracle.attn_int8fp8_from_codes(qc, sq, ks_c, ks_s, vc, sv, idx, L), R)
+    assert e_smooth < 0.75 * e_plain, (e_plain, e_smooth)   # V and P keep their FP8 error
+
+
+def test_quant_k_smooth_rule():
+    # the codes are the INT8 rule applied to fl32(K - m): brute force on one block
+    K = torch.from_numpy(_rand((1, 1, 64, 8), 13, scale=3.0) + 2.0).to(torch.bfloat16)
+    km = oracle.k_channel_mean_ref(K)
+    codes, scales = oracle.quant_k_smooth_ref(K, km)
+    x = K.float().numpy()[0, 0] - km[0, 0][None, :]
+    a = np.float32(np.abs(x).max())
+    inv = np.float32(np.float32(127.0) / a)
+    for t in range(64):
+        for c in range(8):
+            want = int(np.clip(np.rint(np.float32(x[t, c] * inv)), -127, 127))
+            assert codes[0, 0, t, c] == want
+    assert scales[0, 0, 0] == np.float32(a / np.float32(127.0))
