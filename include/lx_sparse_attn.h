@@ -162,6 +162,23 @@ lx_status lx_qk_prologue(const lx_bhld* Q, const lx_bhld* K, const float* wq, co
                          const lx_rope3d* rope, const float* table, const lx_bhld* Yq, const lx_bhld* Yk, float* mq,
                          float* mk, int8_t* qc, float* qs, int8_t* kc, float* ks, cudaStream_t stream);
 
+/* K smoothing -- a variant, not on the pages (the SageAttention family, which
+ * the pages name, subtracts K's mean before quantising).  Subtracting one
+ * vector m from every key shifts each score row by the constant q.m, which the
+ * softmax removes; quantising K - m shrinks the INT8 error when K has large
+ * channel offsets.  Reading: m = the per-(b, h, channel) mean of K over all L
+ * tokens, taken in fp64 and rounded to fp32 once.
+ * lx_k_channel_mean: km fp32 [B,H,D]; ws: scratch of lx_k_channel_mean_ws_size
+ * bytes (8 * B * H * ceil(L/512) * D), 16-byte aligned.  The sums run in a
+ * fixed order, so km is reproducible bit for bit.
+ * lx_quantize_qk_smooth: Q's codes as lx_quantize_qk; K's codes and scales are
+ * those of fl32(K - km) by the same rule.  The attention takes them unchanged
+ * (lx_attn_int8fp8). */
+lx_status lx_k_channel_mean_ws_size(const lx_bhld* K, size_t* bytes);
+lx_status lx_k_channel_mean(const lx_bhld* K, void* ws, size_t ws_bytes, float* km, cudaStream_t stream);
+lx_status lx_quantize_qk_smooth(const lx_bhld* Q, const lx_bhld* K, const float* km, int8_t* qc, float* qs, int8_t* kc,
+                                float* ks, cudaStream_t stream);
+
 /* Step a3 -- FP8 E4M3 V ("600倍加速…", §高效推理算子: "V FP8").
  * vc: uint8 [B,H,L,D] contiguous E4M3 codes; vs: fp32 [B,H,D] scales =
  * absmax over all L tokens / 448 (1 for an all-zero channel);

@@ -159,3 +159,19 @@ def test_prologue_argument_errors_before_launch(lib):
     assert call(outs=[0x20000, 0x30000, 0x40000, None, 0x60000, 0x70000]) == _abi.LX_ERR_INVALID
     assert call(outs=[None, 0x30000, 0x40000, 0x50000, 0x60000, 0x70000]) == _abi.LX_ERR_INVALID
     assert call(outs=[0x20008, 0x30000, 0x40000, 0x50000, 0x60000, 0x70000]) == _abi.LX_ERR_ALIGN
+
+
+def test_smoothing_argument_errors_before_launch(lib):
+    s = ctypes.c_void_p(0)
+    k = _view(L=1000, H=2)
+    n = ctypes.c_size_t()
+    assert lib.lx_k_channel_mean_ws_size(ctypes.byref(k), ctypes.byref(n)) == 0
+    assert n.value == 8 * 1 * 2 * 2 * 128            # ceil(1000 / 512) = 2 spans
+    assert lib.lx_k_channel_mean(ctypes.byref(k), 0x20000, n.value - 8, 0x30000, s) == _abi.LX_ERR_WORKSPACE
+    assert lib.lx_k_channel_mean(ctypes.byref(k), 0x20008, n.value, 0x30000, s) == _abi.LX_ERR_ALIGN
+    assert lib.lx_k_channel_mean(ctypes.byref(k), 0x20000, n.value, None, s) == _abi.LX_ERR_INVALID
+    outs = [0x40000, 0x50000, 0x60000, 0x70000]
+    assert lib.lx_quantize_qk_smooth(ctypes.byref(k), ctypes.byref(k), None, *outs, s) == _abi.LX_ERR_INVALID
+    assert lib.lx_quantize_qk_smooth(ctypes.byref(k), ctypes.byref(k), 0x30008, *outs, s) == _abi.LX_ERR_ALIGN
+    other = _view(L=999, H=2)
+    assert lib.lx_quantize_qk_smooth(ctypes.byref(k), ctypes.byref(other), 0x30000, *outs, s) == _abi.LX_ERR_INVALID

@@ -238,6 +238,42 @@ def lx_qk_prologue_into(Q, K, wq, wk, eps, grid, table, mq, mk, qc=None, qs=None
                               _ptr(kc), _ptr(ks), _stream(stream)), "lx_qk_prologue")
 
 
+def lx_k_channel_mean(K, out=None, ws=None, stream=None):
+    """Per-(b, h, channel) mean of K over all tokens (fp64 sums, fp32 result) [B,H,D]."""
+    lib = _abi.load()
+    B, H, L, D = K.shape
+    k = bhld(K)
+    if out is None:
+        out = torch.empty((B, H, D), dtype=torch.float32, device=K.device)
+    if ws is None:
+        n = ctypes.c_size_t()
+        _check(lib.lx_k_channel_mean_ws_size(ctypes.byref(k), ctypes.byref(n)), "lx_k_channel_mean_ws_size")
+        ws = torch.empty(max(n.value, 16), dtype=torch.uint8, device=K.device)
+    _check(lib.lx_k_channel_mean(ctypes.byref(k), _ptr(ws), ws.numel(), _ptr(out), _stream(stream)),
+           "lx_k_channel_mean")
+    return out
+
+
+def lx_quantize_qk_smooth(Q, K, km=None, out=None, stream=None):
+    """INT8 codes of Q and of K minus its channel means: (qc, qs, kc, ks, km)."""
+    lib = _abi.load()
+    B, H, L, D = Q.shape
+    nB = (L + LX_BLOCK - 1) // LX_BLOCK
+    if km is None:
+        km = lx_k_channel_mean(K, stream=stream)
+    if out is None:
+        dev = Q.device
+        out = (torch.empty((B, H, L, D), dtype=torch.int8, device=dev),
+               torch.empty((B, H, nB), dtype=torch.float32, device=dev),
+               torch.empty((B, H, L, D), dtype=torch.int8, device=dev),
+               torch.empty((B, H, nB), dtype=torch.float32, device=dev))
+    qc, qs, kc, ks = out
+    q, k = bhld(Q), bhld(K)
+    _check(lib.lx_quantize_qk_smooth(ctypes.byref(q), ctypes.byref(k), _ptr(km), _ptr(qc), _ptr(qs), _ptr(kc),
+                                     _ptr(ks), _stream(stream)), "lx_quantize_qk_smooth")
+    return qc, qs, kc, ks, km
+
+
 def lx_quantize_v(V, out=None, amax_ws=None, stream=None):
     lib = _abi.load()
     B, H, L, D = V.shape

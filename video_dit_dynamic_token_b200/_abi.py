@@ -51,6 +51,9 @@ SIGNATURES = {
     "lx_rope3d_table": [_P(LxRope3d), _c_i64, _vp, _vp],
     "lx_qk_prologue": [_P(LxBhld), _P(LxBhld), _vp, _vp, ctypes.c_float, _P(LxRope3d), _vp, _P(LxBhld), _P(LxBhld),
                        _vp, _vp, _vp, _vp, _vp, _vp, _vp],
+    "lx_k_channel_mean_ws_size": [_P(LxBhld), _P(_c_sz)],
+    "lx_k_channel_mean": [_P(LxBhld), _vp, _c_sz, _vp, _vp],
+    "lx_quantize_qk_smooth": [_P(LxBhld), _P(LxBhld), _vp, _vp, _vp, _vp, _vp, _vp],
     "lx_quantize_v": [_P(LxBhld), _vp, _vp, _vp, _vp],
     "lx_quantize_v_noalloc": [_P(LxBhld), _vp, _vp, _vp],
     "lx_attn_bf16": [_P(LxBhld), _P(LxBhld), _P(LxBhld), _P(LxPlan), _P(LxBhld), _vp],

@@ -428,6 +428,54 @@ lx_status lx_qk_prologue(const lx_bhld* Q, const lx_bhld* K, const float* wq, co
                      : launch_qk_pass<64>(Q, K, mq, mk, qc, qs, kc, ks, stream, &pro);
 }
 
+// ---------------------------------------------------------------- K smoothing (variant)
+lx_status lx_k_channel_mean_ws_size(const lx_bhld* K, size_t* bytes) {
+  lx_status st = check_bhld(K);
+  if (st != LX_OK) return st;
+  if (!bytes) return LX_ERR_INVALID;
+  const int64_t nSpan = (K->L + lx::kVSpan - 1) / lx::kVSpan;
+  *bytes = sizeof(double) * (size_t)(K->B * K->H * nSpan * K->D);
+  return LX_OK;
+}
+
+lx_status lx_k_channel_mean(const lx_bhld* K, void* ws, size_t ws_bytes, float* km, cudaStream_t stream) {
+  size_t need = 0;
+  lx_status st = lx_k_channel_mean_ws_size(K, &need);
+  if (st != LX_OK) return st;
+  if (!km) return LX_ERR_INVALID;
+  if (!ws || ws_bytes < need) return LX_ERR_WORKSPACE;
+  if (!al16(ws) || !al16(km)) return LX_ERR_ALIGN;
+  const int64_t BH = K->B * K->H;
+  const int nSpan = (int)((K->L + lx::kVSpan - 1) / lx::kVSpan);
+  double* part = reinterpret_cast<double*>(ws);
+  if (K->D == 128)
+    lx::k_mean_partial_kernel<128><<<(unsigned)(BH * nSpan), 128, 0, stream>>>(view(K), part, (int)K->H, (int)K->L, nSpan);
+  else
+    lx::k_mean_partial_kernel<64><<<(unsigned)(BH * nSpan), 128, 0, stream>>>(view(K), part, (int)K->H, (int)K->L, nSpan);
+  if (cudaGetLastError() != cudaSuccess) return LX_ERR_CUDA;
+  const long long n = BH * K->D;
+  lx::k_mean_final_kernel<<<(unsigned)((n + 255) / 256), 256, 0, stream>>>(part, km, BH, (int)K->D, nSpan, (int)K->L);
+  return launch_status();
+}
+
+lx_status lx_quantize_qk_smooth(const lx_bhld* Q, const lx_bhld* K, const float* km, int8_t* qc, float* qs, int8_t* kc,
+                                float* ks, cudaStream_t stream) {
+  lx_status st;
+  if ((st = check_bhld(Q)) != LX_OK || (st = check_bhld(K)) != LX_OK) return st;
+  if (!same_shape(Q, K) || !km || !qc || !qs || !kc || !ks) return LX_ERR_INVALID;
+  if (!al16(km) || !al16(qc) || !al16(kc) || !al16(qs) || !al16(ks)) return LX_ERR_ALIGN;
+  const int64_t nB = n_blocks(Q->L);
+  dim3 grid((unsigned)(Q->B * Q->H * nB), 2);
+  const lx::ProParams pp{};
+  if (Q->D == 128)
+    lx::qk_block_pass_kernel<128, false, true, false, true><<<grid, 128, 0, stream>>>(
+        view(Q), view(K), nullptr, nullptr, qc, kc, qs, ks, (int)Q->H, (int)Q->L, (int)nB, pp, km);
+  else
+    lx::qk_block_pass_kernel<64, false, true, false, true><<<grid, 128, 0, stream>>>(
+        view(Q), view(K), nullptr, nullptr, qc, kc, qs, ks, (int)Q->H, (int)Q->L, (int)nB, pp, km);
+  return launch_status();
+}
+
 lx_status lx_quantize_v(const lx_bhld* V, uint8_t* vc, float* vs, uint32_t* amax_ws, cudaStream_t stream) {
   lx_status st;
   if ((st = check_bhld(V)) != LX_OK) return st;

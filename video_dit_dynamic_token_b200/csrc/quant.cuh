@@ -94,12 +94,14 @@ struct ProParams {
 // the quantiser and the fused pass share one code path and agree bit for bit.
 // PRO: each valid row is first replaced by the bf16 prologue output (above),
 // so the means and codes are those of that bf16 tensor.
-template <int D, bool MEANS, bool CODES, bool PRO>
+// SMOOTH (K smoothing, a variant not on the pages): K's codes are those of
+// fl32(k - km[b, h, c]) over the block's valid rows, km the channel means of K.
+template <int D, bool MEANS, bool CODES, bool PRO, bool SMOOTH = false>
 __global__ void __launch_bounds__(128) qk_block_pass_kernel(BhldView q, BhldView k, float* __restrict__ mq,
                                                            float* __restrict__ mk, int8_t* __restrict__ qc,
                                                            int8_t* __restrict__ kc, float* __restrict__ qs,
                                                            float* __restrict__ ks, int H, int L, int nB,
-                                                           ProParams pro) {
+                                                           ProParams pro, const float* __restrict__ km = nullptr) {
   constexpr int CH = D / 8;      // 16-byte chunks per row
   constexpr int RG = 128 / CH;   // row groups in the CTA
   constexpr int NR = kBlock / RG;  // rows per thread (= D/16)
@@ -208,17 +210,44 @@ __global__ void __launch_bounds__(128) qk_block_pass_kernel(BhldView q, BhldView
       for (int e = 0; e < 8; ++e) part[warp][c * 8 + e] = a[e];
   }
   float amax = 0.f;
-  if constexpr (CODES) {
-    // |x| maxima on bf16 pairs (exact: widening to fp32 keeps order, and both
-    // maxima ignore a NaN operand as fmaxf does)
-    __nv_bfloat162 m2 = __floats2bfloat162_rn(0.f, 0.f);
+  const bool smooth = SMOOTH && blockIdx.y != 0;
+  float kmv[8];
+  if constexpr (SMOOTH) {
 #pragma unroll
-    for (int i = 0; i < NR; ++i) {
-      const uint32_t w[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
-#pragma unroll
-      for (int e = 0; e < 4; ++e) m2 = __hmax2(m2, __habs2(*reinterpret_cast<const __nv_bfloat162*>(&w[e])));
+    for (int e = 0; e < 8; ++e) kmv[e] = 0.f;
+    if (smooth) {
+      const float4* kmr = reinterpret_cast<const float4*>(km + bh * D + c * 8);
+      const float4 a0 = __ldg(kmr), a1 = __ldg(kmr + 1);
+      kmv[0] = a0.x; kmv[1] = a0.y; kmv[2] = a0.z; kmv[3] = a0.w;
+      kmv[4] = a1.x; kmv[5] = a1.y; kmv[6] = a1.z; kmv[7] = a1.w;
     }
-    amax = fmaxf(__low2float(m2), __high2float(m2));
+  }
+  if constexpr (CODES) {
+    if (smooth) {
+      // |k - km| over the valid rows (the zero-filled rows past L would count |km|)
+#pragma unroll
+      for (int i = 0; i < NR; ++i) {
+        if (r + RG * i < cnt) {
+          const uint32_t w[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            amax = fmaxf(amax, fabsf(bf16lo(w[e]) - kmv[2 * e]));
+            amax = fmaxf(amax, fabsf(bf16hi(w[e]) - kmv[2 * e + 1]));
+          }
+        }
+      }
+    } else {
+      // |x| maxima on bf16 pairs (exact: widening to fp32 keeps order, and both
+      // maxima ignore a NaN operand as fmaxf does)
+      __nv_bfloat162 m2 = __floats2bfloat162_rn(0.f, 0.f);
+#pragma unroll
+      for (int i = 0; i < NR; ++i) {
+        const uint32_t w[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) m2 = __hmax2(m2, __habs2(*reinterpret_cast<const __nv_bfloat162*>(&w[e])));
+      }
+      amax = fmaxf(__low2float(m2), __high2float(m2));
+    }
 #pragma unroll
     for (int off = 16; off; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
     if (lane == 0) red[warp] = amax;
@@ -238,7 +267,22 @@ __global__ void __launch_bounds__(128) qk_block_pass_kernel(BhldView q, BhldView
     int8_t* dst = C + (bh * L + t0 + r) * D + c * 8;
 #pragma unroll
     for (int i = 0; i < NR; ++i) {
-      if (r + RG * i < cnt) *reinterpret_cast<uint2*>(dst + (long long)(RG * i) * D) = i8_codes_x8(v[i], inv);
+      if (r + RG * i < cnt) {
+        uint2 o;
+        if (smooth) {
+          const uint32_t w[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
+          uint32_t t8[8];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            t8[2 * e] = i8_code_bits(bf16lo(w[e]) - kmv[2 * e], inv);
+            t8[2 * e + 1] = i8_code_bits(bf16hi(w[e]) - kmv[2 * e + 1], inv);
+          }
+          o = make_uint2(pack_low_bytes(t8[0], t8[1], t8[2], t8[3]), pack_low_bytes(t8[4], t8[5], t8[6], t8[7]));
+        } else {
+          o = i8_codes_x8(v[i], inv);
+        }
+        *reinterpret_cast<uint2*>(dst + (long long)(RG * i) * D) = o;
+      }
     }
     if (threadIdx.x == 0) {
       float* __restrict__ S = blockIdx.y == 0 ? qs : ks;
@@ -360,6 +404,56 @@ __global__ void __launch_bounds__(128, 4) v_quant_kernel(BhldView v, const uint3
     bh = bhn;
     blk = blkn;
   }
+}
+
+// ---------------------------------------------------------------------------
+// K channel means for K smoothing (a variant not on the pages), in two
+// deterministic passes: one 128-thread CTA per (b*h, 512-token span) sums its
+// rows per channel in fp64 (lanes on 16-byte chunks, rows in order, then the
+// row groups in order through shared memory); then one thread per (b*h,
+// channel) adds the spans in order, divides by L and rounds to fp32 once.
+template <int D>
+__global__ void __launch_bounds__(128) k_mean_partial_kernel(BhldView k, double* __restrict__ part, int H, int L,
+                                                            int nSpan) {
+  constexpr int CH = D / 8;
+  constexpr int RPP = 128 / CH;
+  const long long bh = blockIdx.x / nSpan;
+  const int span = (int)(blockIdx.x - bh * nSpan);
+  const long long b = bh / H, h = bh - b * H;
+  const int c = threadIdx.x % CH, r0 = threadIdx.x / CH;
+  const int t_begin = span * kVSpan, t_end = min(L, t_begin + kVSpan);
+  double s[8] = {0., 0., 0., 0., 0., 0., 0., 0.};
+  const __nv_bfloat16* base = k.p + b * k.sB + h * k.sH + c * 8;
+  for (int t = t_begin + r0; t < t_end; t += RPP) {
+    const uint4 x = ld_stream_v4(base + (long long)t * k.sL);
+    const uint32_t w[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      s[2 * e] += (double)bf16lo(w[e]);
+      s[2 * e + 1] += (double)bf16hi(w[e]);
+    }
+  }
+  __shared__ double red[128][9];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) red[threadIdx.x][e] = s[e];
+  __syncthreads();
+  if (threadIdx.x < D) {
+    const int ch = threadIdx.x / 8, e = threadIdx.x % 8;
+    double acc = 0.;
+    for (int rr = 0; rr < RPP; ++rr) acc += red[rr * CH + ch][e];
+    part[((long long)bh * nSpan + span) * D + threadIdx.x] = acc;
+  }
+}
+
+__global__ void k_mean_final_kernel(const double* __restrict__ part, float* __restrict__ km, long long BH, int D,
+                                    int nSpan, int L) {
+  const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= BH * D) return;
+  const long long bh = i / D;
+  const int ch = (int)(i - bh * D);
+  double acc = 0.;
+  for (int sp = 0; sp < nSpan; ++sp) acc += part[(bh * nSpan + sp) * D + ch];
+  km[i] = (float)(acc / (double)L);
 }
 
 // ---------------------------------------------------------------------------
