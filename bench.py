@@ -161,6 +161,10 @@ def run_ours(args, rank, world, local_rank):
         names = ["pool_quant_qk", "score_topk", "quant_v", "attn"]
         if args.prologue:
             names[0] = "qk_prologue"
+        elif args.smooth_k:
+            # K channel means (two launches), then the Q/K pass with K smoothed
+            launches_per_step = 8
+            names = ["k_mean", "pool_quant_qk_smooth", "score_topk", "quant_v", "attn"]
     else:
         launches_per_step = 4  # pool, score GEMM, top-k, attention
         names = ["pool", "score_topk", "attn"]
@@ -174,6 +178,11 @@ def run_ours(args, rank, world, local_rank):
         wk = (1.0 + 0.2 * torch.randn(H, d, generator=g)).float().to(dev)
         pro = dict(wq=wq, wk=wk, table=lx.lx_rope3d_table(w.grid, d, device=dev))
 
+    km_buf = km_ws = None
+    if args.smooth_k and mode == "int8fp8":
+        km_buf = torch.empty((B, H, d), dtype=torch.float32, device=dev)
+        km_ws = torch.empty(8 * B * H * ((L + 511) // 512) * d, dtype=torch.uint8, device=dev)
+
     def step(ev=None):
         marks = iter(range(len(names) + 1))
         def mark():
@@ -181,7 +190,11 @@ def run_ours(args, rank, world, local_rank):
             if ev is not None:
                 ev[i].record(stream)
         mark()
-        if pro is not None:
+        if args.smooth_k and mode == "int8fp8":
+            lx.lx_k_channel_mean(K, out=km_buf, ws=km_ws)
+            mark()
+            lx.lx_pool_quantize_qk_smooth(Q, K, km_buf, (mq, mk, qc, qs, kc, ks))
+        elif pro is not None:
             lx.lx_qk_prologue_into(Q, K, pro["wq"], pro["wk"], 1e-6, w.grid, pro["table"], mq, mk, qc, qs, kc, ks)
         elif mode == "int8fp8":
             lx.lx_pool_quantize_qk(Q, K, out=(mq, mk, qc, qs, kc, ks))
@@ -274,7 +287,10 @@ def run_ours(args, rank, world, local_rank):
     plan_out_b = B * H * nB * k * 4 + B * H * nB * ((nB + 31) // 32) * 4
     phase_bytes = {"score_topk": means_b + plan_out_b}
     if mode == "int8fp8":
-        phase_bytes[names[0]] = 2 * N * 2 + 2 * N + means_b + 2 * B * H * nB * 4
+        qk_name = "pool_quant_qk_smooth" if args.smooth_k else names[0]
+        phase_bytes[qk_name] = 2 * N * 2 + 2 * N + means_b + 2 * B * H * nB * 4
+        if args.smooth_k:
+            phase_bytes["k_mean"] = N * 2 + B * H * d * 4  # K read once
         phase_bytes["quant_v"] = 2 * N * 2 + N + B * H * d * 4  # V read twice: the channel scale needs all of V
     else:
         phase_bytes["pool"] = 2 * N * 2 + means_b
@@ -390,6 +406,8 @@ def main():
                     help="grid shape (the headline is 720p; the others are characterisation runs)")
     ap.add_argument("--mode", default=MODE, choices=["int8fp8", "bf16"])
     ap.add_argument("--keep", type=float, default=0.0, help="override the workload's keep ratio (sweeps)")
+    ap.add_argument("--smooth-k", action="store_true",
+                    help="int8fp8: K smoothing (channel means of K subtracted before its INT8 codes)")
     ap.add_argument("--prologue", action="store_true",
                     help="int8fp8: the Q/K pass also applies per-head RMSNorm and 3D RoPE (lx_qk_prologue)")
     args = ap.parse_args()

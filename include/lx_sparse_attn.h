@@ -178,6 +178,10 @@ lx_status lx_k_channel_mean_ws_size(const lx_bhld* K, size_t* bytes);
 lx_status lx_k_channel_mean(const lx_bhld* K, void* ws, size_t ws_bytes, float* km, cudaStream_t stream);
 lx_status lx_quantize_qk_smooth(const lx_bhld* Q, const lx_bhld* K, const float* km, int8_t* qc, float* qs, int8_t* kc,
                                 float* ks, cudaStream_t stream);
+/* The same codes plus the block means of Q and K (of the unshifted K, which
+ * rank the key blocks alike) in one read, as lx_pool_quantize_qk. */
+lx_status lx_pool_quantize_qk_smooth(const lx_bhld* Q, const lx_bhld* K, const float* km, float* mq, float* mk,
+                                     int8_t* qc, float* qs, int8_t* kc, float* ks, cudaStream_t stream);
 
 /* Step a3 -- FP8 E4M3 V ("600倍加速…", §高效推理算子: "V FP8").
  * vc: uint8 [B,H,L,D] contiguous E4M3 codes; vs: fp32 [B,H,D] scales =

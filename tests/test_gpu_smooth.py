@@ -79,3 +79,20 @@ def test_smoothing_reduces_error_on_offset_keys():
     _, e_plain = compare_rows(O_plain, R, L, blocks)
     _, e_smooth = compare_rows(O_smooth, R, L, blocks)
     assert e_smooth < 0.75 * e_plain, (e_plain, e_smooth)
+
+
+def test_fused_means_and_smoothed_codes_equal_separate_calls():
+    Q, K, _ = _offset_qkv(1, 2, 2500, 128, seed=23, offset=5.0)
+    km = lx.lx_k_channel_mean(K)
+    B, H, L, d = Q.shape
+    nB = oracle.n_blocks(L)
+    out = (torch.empty((B, H, nB, d), dtype=torch.float32, device=DEV),
+           torch.empty((B, H, nB, d), dtype=torch.float32, device=DEV),
+           torch.empty((B, H, L, d), dtype=torch.int8, device=DEV), torch.empty((B, H, nB), dtype=torch.float32, device=DEV),
+           torch.empty((B, H, L, d), dtype=torch.int8, device=DEV), torch.empty((B, H, nB), dtype=torch.float32, device=DEV))
+    lx.lx_pool_quantize_qk_smooth(Q, K, km, out)
+    pq, pk = lx.lx_pool_means(Q, K)
+    qc, qs, kc, ks, _ = lx.lx_quantize_qk_smooth(Q, K, km)
+    torch.cuda.synchronize()
+    for a, b in zip(out, (pq, pk, qc, qs, kc, ks)):
+        assert torch.equal(a, b)

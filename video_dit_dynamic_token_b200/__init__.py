@@ -274,6 +274,16 @@ def lx_quantize_qk_smooth(Q, K, km=None, out=None, stream=None):
     return qc, qs, kc, ks, km
 
 
+def lx_pool_quantize_qk_smooth(Q, K, km, out, stream=None):
+    """Block means of Q and K and INT8 codes of Q and K - km, into out = (mq, mk, qc, qs, kc, ks)."""
+    lib = _abi.load()
+    mq, mk, qc, qs, kc, ks = out
+    q, k = bhld(Q), bhld(K)
+    _check(lib.lx_pool_quantize_qk_smooth(ctypes.byref(q), ctypes.byref(k), _ptr(km), _ptr(mq), _ptr(mk), _ptr(qc),
+                                          _ptr(qs), _ptr(kc), _ptr(ks), _stream(stream)), "lx_pool_quantize_qk_smooth")
+    return out
+
+
 def lx_quantize_v(V, out=None, amax_ws=None, stream=None):
     lib = _abi.load()
     B, H, L, D = V.shape

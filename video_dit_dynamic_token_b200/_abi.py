@@ -54,6 +54,7 @@ SIGNATURES = {
     "lx_k_channel_mean_ws_size": [_P(LxBhld), _P(_c_sz)],
     "lx_k_channel_mean": [_P(LxBhld), _vp, _c_sz, _vp, _vp],
     "lx_quantize_qk_smooth": [_P(LxBhld), _P(LxBhld), _vp, _vp, _vp, _vp, _vp, _vp],
+    "lx_pool_quantize_qk_smooth": [_P(LxBhld), _P(LxBhld), _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp],
     "lx_quantize_v": [_P(LxBhld), _vp, _vp, _vp, _vp],
     "lx_quantize_v_noalloc": [_P(LxBhld), _vp, _vp, _vp],
     "lx_attn_bf16": [_P(LxBhld), _P(LxBhld), _P(LxBhld), _P(LxPlan), _P(LxBhld), _vp],

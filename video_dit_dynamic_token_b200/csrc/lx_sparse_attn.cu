@@ -165,6 +165,14 @@ lx_status launch_score(const float* mq, const float* mk, int64_t BH, int64_t nB,
   return launch_status();
 }
 
+template <int D, bool MEANS>
+void launch_smooth(const lx_bhld* Q, const lx_bhld* K, const float* km, float* mq, float* mk, int8_t* qc, float* qs,
+                   int8_t* kc, float* ks, cudaStream_t s) {
+  const int64_t nB = n_blocks(Q->L);
+  dim3 grid((unsigned)(Q->B * Q->H * nB), 2);
+  lx::qk_block_pass_kernel<D, MEANS, true, false, true><<<grid, 128, 0, s>>>(
+      view(Q), view(K), mq, mk, qc, kc, qs, ks, (int)Q->H, (int)Q->L, (int)nB, lx::ProParams{}, km);
+}
 template <int D>
 lx_status launch_quant_v(const lx_bhld* V, uint8_t* vc, float* vs, uint32_t* amax, cudaStream_t s) {
   const int64_t BH = V->B * V->H, nB = n_blocks(V->L);
@@ -464,15 +472,23 @@ lx_status lx_quantize_qk_smooth(const lx_bhld* Q, const lx_bhld* K, const float*
   if ((st = check_bhld(Q)) != LX_OK || (st = check_bhld(K)) != LX_OK) return st;
   if (!same_shape(Q, K) || !km || !qc || !qs || !kc || !ks) return LX_ERR_INVALID;
   if (!al16(km) || !al16(qc) || !al16(kc) || !al16(qs) || !al16(ks)) return LX_ERR_ALIGN;
-  const int64_t nB = n_blocks(Q->L);
-  dim3 grid((unsigned)(Q->B * Q->H * nB), 2);
-  const lx::ProParams pp{};
   if (Q->D == 128)
-    lx::qk_block_pass_kernel<128, false, true, false, true><<<grid, 128, 0, stream>>>(
-        view(Q), view(K), nullptr, nullptr, qc, kc, qs, ks, (int)Q->H, (int)Q->L, (int)nB, pp, km);
+    launch_smooth<128, false>(Q, K, km, nullptr, nullptr, qc, qs, kc, ks, stream);
   else
-    lx::qk_block_pass_kernel<64, false, true, false, true><<<grid, 128, 0, stream>>>(
-        view(Q), view(K), nullptr, nullptr, qc, kc, qs, ks, (int)Q->H, (int)Q->L, (int)nB, pp, km);
+    launch_smooth<64, false>(Q, K, km, nullptr, nullptr, qc, qs, kc, ks, stream);
+  return launch_status();
+}
+
+lx_status lx_pool_quantize_qk_smooth(const lx_bhld* Q, const lx_bhld* K, const float* km, float* mq, float* mk,
+                                     int8_t* qc, float* qs, int8_t* kc, float* ks, cudaStream_t stream) {
+  lx_status st;
+  if ((st = check_bhld(Q)) != LX_OK || (st = check_bhld(K)) != LX_OK) return st;
+  if (!same_shape(Q, K) || !km || !mq || !mk || !qc || !qs || !kc || !ks) return LX_ERR_INVALID;
+  if (!al16(km) || !al16(mq) || !al16(mk) || !al16(qc) || !al16(kc) || !al16(qs) || !al16(ks)) return LX_ERR_ALIGN;
+  if (Q->D == 128)
+    launch_smooth<128, true>(Q, K, km, mq, mk, qc, qs, kc, ks, stream);
+  else
+    launch_smooth<64, true>(Q, K, km, mq, mk, qc, qs, kc, ks, stream);
   return launch_status();
 }
 
