@@ -141,3 +141,16 @@ def test_plan_narrow_score_range_with_large_offset():
         plan = lx.lx_sparse_attn_plan(Q, K, keep)
         assert lx.lx_last_device_status() == 0
         check_plan(plan.idx, plan.mask, Q.cpu(), K.cpu(), keep)
+
+
+@pytest.mark.parametrize("smooth", [True, False])
+def test_plan_parity_maximum_row_length(smooth):
+    # nB = 2176, the longest score row the selection holds (17 chunks of 128),
+    # on a grid of 2 heads; ragged last tile of the score GEMM (2176 = 17 * 128)
+    grid = (17, 64, 128)    # 139264 tokens = 2176 blocks of 64
+    Q, K, _ = synth.make_qkv(1, 2, 128, grid, seed=4, smooth=smooth, device=DEV)
+    assert Q.shape[2] == 64 * 2176
+    plan = lx.lx_sparse_attn_plan(Q, K, 0.1)
+    assert lx.lx_last_device_status() == 0
+    assert plan.nB == 2176
+    check_plan(plan.idx, plan.mask, Q.cpu(), K.cpu(), 0.1)
