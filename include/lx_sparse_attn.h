@@ -240,6 +240,16 @@ lx_status lx_fwd_workspace_size(const lx_bhld* Q, lx_mode mode, size_t* bytes);
 lx_status lx_sparse_attn_fwd(const lx_bhld* Q, const lx_bhld* K, const lx_bhld* V, const lx_plan* plan, lx_mode mode,
                              const lx_bhld* O, void* ws, size_t ws_bytes, cudaStream_t stream);
 
+/* Steps a1-a4 in one call: plan (written to *plan, whose idx/mask the caller
+ * sets as for lx_score_topk) and forward.  INT8/FP8 mode reads Q and K once
+ * for the block means and the INT8 codes (lx_pool_quantize_qk), so the result
+ * equals lx_sparse_attn_plan followed by lx_sparse_attn_fwd bit for bit with
+ * one pass over Q and K fewer.  ws: lx_sparse_attn_ws_size bytes, 256-byte
+ * aligned (the planner's workspace, rounded to 256, then the forward's). */
+lx_status lx_sparse_attn_ws_size(const lx_bhld* Q, double keep, lx_mode mode, size_t* bytes);
+lx_status lx_sparse_attn(const lx_bhld* Q, const lx_bhld* K, const lx_bhld* V, double keep, lx_mode mode,
+                         lx_plan* plan, const lx_bhld* O, void* ws, size_t ws_bytes, cudaStream_t stream);
+
 /* Synchronises `stream`, returns and clears the device status word of the
  * current device: LX_OK, LX_ERR_TIMEOUT, LX_ERR_PLAN, or LX_ERR_CUDA when the
  * stream itself reports an error. */

@@ -140,3 +140,16 @@ def test_attn_int8fp8_large_qk_scales(qk_scale):
     R = oracle.attn_ref_int8fp8(Q.cpu(), K.cpu(), V.cpu(), ref["idx"])
     mx, rl1 = compare_rows(O, R, L, _all_blocks(B, H, L))
     assert mx <= TOL_I8_MAXABS and rl1 <= TOL_I8_RELL1, (mx, rl1)
+
+
+@pytest.mark.parametrize("mode", ["int8fp8", "bf16"])
+def test_one_call_equals_plan_then_forward(mode):
+    B, H, L, d, keep = 1, 3, 5000, 128, 0.15
+    Q, K, V = synth.random_qkv(B, H, L, d, seed=41, scale=1.5, device=DEV)
+    plan = lx.lx_sparse_attn_plan(Q, K, keep)
+    O1 = lx.lx_sparse_attn_fwd(Q, K, V, plan, mode)
+    O2, plan2 = lx.lx_sparse_attn(Q, K, V, keep, mode)
+    torch.cuda.synchronize()
+    assert lx.lx_last_device_status() == 0
+    assert torch.equal(plan.idx, plan2.idx) and torch.equal(plan.mask, plan2.mask)
+    assert torch.equal(O1, O2)

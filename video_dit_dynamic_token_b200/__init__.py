@@ -351,6 +351,32 @@ def lx_sparse_attn_fwd(Q, K, V, plan: Plan, mode="int8fp8", out=None, ws=None, s
     return out
 
 
+def lx_sparse_attn_ws_size(Q, keep, mode="int8fp8") -> int:
+    lib = _abi.load()
+    n = ctypes.c_size_t()
+    q = bhld(Q)
+    _check(lib.lx_sparse_attn_ws_size(ctypes.byref(q), float(keep), MODES[mode], ctypes.byref(n)),
+           "lx_sparse_attn_ws_size")
+    return n.value
+
+
+def lx_sparse_attn(Q, K, V, keep, mode="int8fp8", plan: Plan | None = None, out=None, ws=None, stream=None):
+    """Plan and forward in one call (Q and K read once for means and codes): (O, plan)."""
+    lib = _abi.load()
+    B, H, L, D = Q.shape
+    if plan is None:
+        plan = empty_plan(B, H, L, D, keep, Q.device)
+    if out is None:
+        out = torch.empty_like(Q)
+    if ws is None:
+        ws = torch.empty(max(lx_sparse_attn_ws_size(Q, keep, mode), 256), dtype=torch.uint8, device=Q.device)
+    q, k, v, o, cp = bhld(Q), bhld(K), bhld(V), bhld(out), plan.c()
+    _check(lib.lx_sparse_attn(ctypes.byref(q), ctypes.byref(k), ctypes.byref(v), float(keep), MODES[mode],
+                              ctypes.byref(cp), ctypes.byref(o), _ptr(ws), ws.numel(), _stream(stream)),
+           "lx_sparse_attn")
+    return out, plan
+
+
 def lx_last_device_status(stream=None) -> int:
     return _abi.load().lx_last_device_status(_stream(stream))
 

@@ -61,6 +61,8 @@ SIGNATURES = {
     "lx_attn_int8fp8": [_vp, _vp, _vp, _vp, _vp, _vp, _P(LxPlan), _P(LxBhld), _vp],
     "lx_fwd_workspace_size": [_P(LxBhld), ctypes.c_int, _P(_c_sz)],
     "lx_sparse_attn_fwd": [_P(LxBhld), _P(LxBhld), _P(LxBhld), _P(LxPlan), ctypes.c_int, _P(LxBhld), _vp, _c_sz, _vp],
+    "lx_sparse_attn_ws_size": [_P(LxBhld), _dbl, ctypes.c_int, _P(_c_sz)],
+    "lx_sparse_attn": [_P(LxBhld), _P(LxBhld), _P(LxBhld), _dbl, ctypes.c_int, _P(LxPlan), _P(LxBhld), _vp, _c_sz, _vp],
     "lx_last_device_status": [_vp],
     "lx_debug_wait_timeout": [_u64, _vp],
     "lx_status_string": [ctypes.c_int],

@@ -597,6 +597,58 @@ lx_status lx_sparse_attn_fwd(const lx_bhld* Q, const lx_bhld* K, const lx_bhld* 
   return lx_attn_int8fp8(qc, qs, kc, ks, vc, vs, plan, O, stream);
 }
 
+lx_status lx_sparse_attn_ws_size(const lx_bhld* Q, double keep, lx_mode mode, size_t* bytes) {
+  if (!Q || !bytes) return LX_ERR_INVALID;
+  size_t plan_ws = 0, fwd_ws = 0;
+  lx_status st = lx_plan_size(Q->B, Q->H, Q->L, Q->D, keep, nullptr, nullptr, nullptr, &plan_ws);
+  if (st != LX_OK) return st;
+  if ((st = lx_fwd_workspace_size(Q, mode, &fwd_ws)) != LX_OK) return st;
+  *bytes = align256(plan_ws) + fwd_ws;
+  return LX_OK;
+}
+
+lx_status lx_sparse_attn(const lx_bhld* Q, const lx_bhld* K, const lx_bhld* V, double keep, lx_mode mode,
+                         lx_plan* plan, const lx_bhld* O, void* ws, size_t ws_bytes, cudaStream_t stream) {
+  lx_status st;
+  if ((st = check_bhld(Q)) != LX_OK || (st = check_bhld(K)) != LX_OK || (st = check_bhld(V)) != LX_OK ||
+      (st = check_bhld(O)) != LX_OK)
+    return st;
+  if (!same_shape(Q, K) || !same_shape(Q, V) || !same_shape(Q, O) || !plan) return LX_ERR_INVALID;
+  if (mode != LX_MODE_BF16 && mode != LX_MODE_INT8FP8) return LX_ERR_INVALID;
+  size_t need = 0, plan_ws = 0;
+  if ((st = lx_sparse_attn_ws_size(Q, keep, mode, &need)) != LX_OK) return st;
+  if ((st = lx_plan_size(Q->B, Q->H, Q->L, Q->D, keep, nullptr, nullptr, nullptr, &plan_ws)) != LX_OK) return st;
+  if (!ws || ws_bytes < need) return LX_ERR_WORKSPACE;
+  if ((reinterpret_cast<uintptr_t>(ws) & 255u) != 0) return LX_ERR_ALIGN;
+  if (n_blocks(Q->L) > kMaxPlannerNB) return LX_ERR_UNSUPPORTED;
+  // workspace: [means of Q | means of K | scores (planner) | codes and scales (forward)]
+  char* base = reinterpret_cast<char*>(ws);
+  const size_t means = align256(sizeof(float) * (size_t)(Q->B * Q->H * n_blocks(Q->L) * Q->D));
+  float* mq = reinterpret_cast<float*>(base);
+  float* mk = reinterpret_cast<float*>(base + means);
+  char* sc = base + 2 * means;
+  const size_t sc_bytes = plan_ws - 2 * means;
+  if (mode == LX_MODE_BF16) {
+    if ((st = lx_pool_means(Q, K, mq, mk, stream)) != LX_OK) return st;
+    if ((st = lx_score_topk(mq, mk, Q->B, Q->H, Q->L, Q->D, keep, plan, sc, sc_bytes, stream)) != LX_OK) return st;
+    return lx_attn_bf16(Q, K, V, plan, O, stream);
+  }
+  const FwdWs w = fwd_layout(Q);
+  char* fb = base + align256(plan_ws);
+  int8_t* qc = reinterpret_cast<int8_t*>(fb + w.qc);
+  int8_t* kc = reinterpret_cast<int8_t*>(fb + w.kc);
+  uint8_t* vc = reinterpret_cast<uint8_t*>(fb + w.vc);
+  float* qs = reinterpret_cast<float*>(fb + w.qs);
+  float* ks = reinterpret_cast<float*>(fb + w.ks);
+  float* vs = reinterpret_cast<float*>(fb + w.vs);
+  uint32_t* amax = reinterpret_cast<uint32_t*>(fb + w.amax);
+  // Q and K are read once for the block means and the INT8 codes
+  if ((st = lx_pool_quantize_qk(Q, K, mq, mk, qc, qs, kc, ks, stream)) != LX_OK) return st;
+  if ((st = lx_score_topk(mq, mk, Q->B, Q->H, Q->L, Q->D, keep, plan, sc, sc_bytes, stream)) != LX_OK) return st;
+  if ((st = lx_quantize_v(V, vc, vs, amax, stream)) != LX_OK) return st;
+  return lx_attn_int8fp8(qc, qs, kc, ks, vc, vs, plan, O, stream);
+}
+
 lx_status lx_last_device_status(cudaStream_t stream) {
   if (cudaStreamSynchronize(stream) != cudaSuccess) return LX_ERR_CUDA;
   int v = 0;

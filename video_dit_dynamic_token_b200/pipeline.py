@@ -13,7 +13,7 @@ from __future__ import annotations
 
 import torch
 
-from . import empty_plan, lx_fwd_workspace_size, lx_plan_size, lx_sparse_attn_fwd, lx_sparse_attn_plan
+from . import empty_plan, lx_sparse_attn, lx_sparse_attn_ws_size
 
 
 class HostPipeline:
@@ -34,12 +34,10 @@ class HostPipeline:
         self.slots = []
         for _ in range(2):
             q, k, v, o = (torch.empty(shape, dtype=torch.bfloat16, device=self.dev) for _ in range(4))
-            _, _, _, wb = lx_plan_size(B, self.hc, L, D, keep)
-            ws_plan = torch.empty(max(wb, 256), dtype=torch.uint8, device=self.dev)
-            ws_fwd = torch.empty(max(lx_fwd_workspace_size(q, mode), 256), dtype=torch.uint8, device=self.dev)
+            ws = torch.empty(max(lx_sparse_attn_ws_size(q, keep, mode), 256), dtype=torch.uint8, device=self.dev)
             # one plan per distinct chunk width (the last chunk may be narrower)
             plans = {n: empty_plan(B, n, L, D, keep, self.dev) for n in {h1 - h0 for h0, h1 in self.chunks}}
-            self.slots.append(dict(q=q, k=k, v=v, o=o, ws_plan=ws_plan, ws_fwd=ws_fwd, plans=plans))
+            self.slots.append(dict(q=q, k=k, v=v, o=o, ws=ws, plans=plans))
         self.s_h2d = torch.cuda.Stream(self.dev)
         self.s_cmp = torch.cuda.Stream(self.dev)
         self.s_d2h = torch.cuda.Stream(self.dev)
@@ -69,8 +67,8 @@ class HostPipeline:
             if c >= 2:
                 self.s_cmp.wait_event(ev_d2h[c - 2])
             with torch.cuda.stream(self.s_cmp):
-                plan = lx_sparse_attn_plan(dq, dk, self.keep, plan=sl["plans"][n], ws=sl["ws_plan"], stream=self.s_cmp)
-                lx_sparse_attn_fwd(dq, dk, dv, plan, self.mode, out=do, ws=sl["ws_fwd"], stream=self.s_cmp)
+                lx_sparse_attn(dq, dk, dv, self.keep, self.mode, plan=sl["plans"][n], out=do, ws=sl["ws"],
+                               stream=self.s_cmp)
                 e_cmp.record(self.s_cmp)
             self.s_d2h.wait_event(e_cmp)
             with torch.cuda.stream(self.s_d2h):
