@@ -11,3 +11,5 @@ from .sparse_attn_ref import (BLOCK, E4M3_MAX, attn_int8fp8_from_codes, attn_ref
                               rel_l1_err, select_topk)
 from .prologue_ref import (ROPE_THETA, bf16_round, k_channel_mean_ref, prologue_ref,  # noqa: F401
                            qk_rmsnorm_ref, quant_k_smooth_ref, rope3d_ref, rope3d_split, token_positions)
+from .ulysses_ref import (all_to_all_ref, fp8_rows_dequant_ref, fp8_rows_ref, pack_o_ref, pack_qkv_ref,  # noqa: F401
+                          unpack_o_ref, unpack_qkv_ref)
