@@ -183,6 +183,38 @@ lx_status lx_quantize_qk_smooth(const lx_bhld* Q, const lx_bhld* K, const float*
 lx_status lx_pool_quantize_qk_smooth(const lx_bhld* Q, const lx_bhld* K, const float* km, float* mq, float* mk,
                                      int8_t* qc, float* qs, int8_t* kc, float* ks, cudaStream_t stream);
 
+/* Light-Ulysses exchange (multi-GPU sequence parallelism, "600倍加速…",
+ * §多卡路径: the sequence is split over the GPUs and an all-to-all moves the
+ * data between the sequence and head dimensions; FP8 payloads, Q/K/V fused in
+ * one payload, the exchange run per head chunk).  Reading: rank r holds tokens
+ * [r Lr, (r+1) Lr) of all H heads before the exchange, heads [r Hr, (r+1) Hr)
+ * (Hr = H / N) of all L = N Lr tokens after it.  One FP8 scale per (token,
+ * head, tensor) row of D values: s = absmax/448 (1 for an all-zero row), code
+ * = E4M3_rn_satfinite(fl32(x * fl32(448/absmax))); the receiver writes
+ * bf16(fl32(decode(code) * s)).  The collective itself is the caller's (one
+ * all-to-all with equal splits over the leading N of each buffer); these calls
+ * build and read its buffers.
+ *
+ * lx_ulysses_pack_qkv: q, k, v this rank's shard viewed as [B, H, Lr, D] (any
+ * strides, e.g. the [B, Lr, H, D] layout); sends heads h0 .. h0+hc-1 of each
+ * destination's range: codes [N][B][hc][Lr][3][D] uint8, scales
+ * [N][B][hc][Lr][3] fp32.
+ * lx_ulysses_unpack_qkv: the received buffers (same layout, slice n from rank
+ * n) into q, k, v [B, hc, L, D] (L divisible by N; token n Lr + t from rank n).
+ * lx_ulysses_pack_o: the attention output o [B, hc, L, D] of those heads:
+ * codes [N][B][hc][Lr][D], scales [N][B][hc][Lr], slice n holding rank n's
+ * tokens.
+ * lx_ulysses_unpack_o: the received output buffers into this rank's shard
+ * out [B, H, Lr, D] (any strides), heads n Hr + h0 .. n Hr + h0 + hc - 1 from
+ * rank n.  Pointers 16-byte aligned; errors as elsewhere. */
+lx_status lx_ulysses_pack_qkv(const lx_bhld* q, const lx_bhld* k, const lx_bhld* v, int64_t N, int64_t h0, int64_t hc,
+                              uint8_t* codes, float* scales, cudaStream_t stream);
+lx_status lx_ulysses_unpack_qkv(const uint8_t* codes, const float* scales, int64_t N, const lx_bhld* q,
+                                const lx_bhld* k, const lx_bhld* v, cudaStream_t stream);
+lx_status lx_ulysses_pack_o(const lx_bhld* o, int64_t N, uint8_t* codes, float* scales, cudaStream_t stream);
+lx_status lx_ulysses_unpack_o(const uint8_t* codes, const float* scales, int64_t N, int64_t h0, int64_t hc,
+                              const lx_bhld* out, cudaStream_t stream);
+
 /* Step a3 -- FP8 E4M3 V ("600倍加速…", §高效推理算子: "V FP8").
  * vc: uint8 [B,H,L,D] contiguous E4M3 codes; vs: fp32 [B,H,D] scales =
  * absmax over all L tokens / 448 (1 for an all-zero channel);

@@ -63,6 +63,10 @@ SIGNATURES = {
     "lx_sparse_attn_fwd": [_P(LxBhld), _P(LxBhld), _P(LxBhld), _P(LxPlan), ctypes.c_int, _P(LxBhld), _vp, _c_sz, _vp],
     "lx_sparse_attn_ws_size": [_P(LxBhld), _dbl, ctypes.c_int, _P(_c_sz)],
     "lx_sparse_attn": [_P(LxBhld), _P(LxBhld), _P(LxBhld), _dbl, ctypes.c_int, _P(LxPlan), _P(LxBhld), _vp, _c_sz, _vp],
+    "lx_ulysses_pack_qkv": [_P(LxBhld), _P(LxBhld), _P(LxBhld), _c_i64, _c_i64, _c_i64, _vp, _vp, _vp],
+    "lx_ulysses_unpack_qkv": [_vp, _vp, _c_i64, _P(LxBhld), _P(LxBhld), _P(LxBhld), _vp],
+    "lx_ulysses_pack_o": [_P(LxBhld), _c_i64, _vp, _vp, _vp],
+    "lx_ulysses_unpack_o": [_vp, _vp, _c_i64, _c_i64, _c_i64, _P(LxBhld), _vp],
     "lx_last_device_status": [_vp],
     "lx_debug_wait_timeout": [_u64, _vp],
     "lx_status_string": [ctypes.c_int],

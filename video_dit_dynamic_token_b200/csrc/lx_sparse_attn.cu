@@ -11,6 +11,7 @@
 #include "ptx.cuh"
 #include "planner.cuh"
 #include "quant.cuh"
+#include "ulysses.cuh"
 #include "attn.cuh"
 
 namespace {
@@ -265,6 +266,24 @@ FwdWs fwd_layout(const lx_bhld* Q) {
 }  // namespace
 
 // ====================================================================== C ABI
+// Light-Ulysses launch helper (the entries are below, in the C block)
+namespace {
+lx::BhldRW rw(const lx_bhld* t) {
+  return lx::BhldRW{reinterpret_cast<__nv_bfloat16*>(t->data), t->sB, t->sH, t->sL};
+}
+template <int MODE>
+lx_status launch_ulysses(lx::UlyssesArgs a, int64_t D, cudaStream_t s) {
+  if (a.rows == 0) return LX_OK;
+  const long long threads = a.rows * (D / 8);
+  const unsigned blocks = (unsigned)((threads + 255) / 256);
+  if (D == 128)
+    lx::ulysses_rows_kernel<128, MODE><<<blocks, 256, 0, s>>>(a);
+  else
+    lx::ulysses_rows_kernel<64, MODE><<<blocks, 256, 0, s>>>(a);
+  return launch_status();
+}
+}  // namespace
+
 extern "C" {
 
 const char* lx_status_string(lx_status st) {
@@ -663,6 +682,91 @@ lx_status lx_debug_wait_timeout(uint64_t limit_ns, cudaStream_t stream) {
   if (limit_ns == 0 || limit_ns > 10000000000ull) return LX_ERR_INVALID;
   lx::wait_timeout_probe_kernel<<<1, 32, 0, stream>>>((unsigned long long)limit_ns);
   return launch_status();
+}
+
+// ---------------------------------------------------------------- Light-Ulysses exchange
+lx_status lx_ulysses_pack_qkv(const lx_bhld* q, const lx_bhld* k, const lx_bhld* v, int64_t N, int64_t h0, int64_t hc,
+                              uint8_t* codes, float* scales, cudaStream_t stream) {
+  lx_status st;
+  if ((st = check_bhld(q)) != LX_OK || (st = check_bhld(k)) != LX_OK || (st = check_bhld(v)) != LX_OK) return st;
+  if (!same_shape(q, k) || !same_shape(q, v) || !codes || !scales) return LX_ERR_INVALID;
+  if (N < 1 || q->H % N != 0 || h0 < 0 || hc < 1 || h0 + hc > q->H / N) return LX_ERR_INVALID;
+  if (!al16(codes) || !al16(scales)) return LX_ERR_ALIGN;
+  lx::UlyssesArgs a{};
+  a.x[0] = rw(q);
+  a.x[1] = rw(k);
+  a.x[2] = rw(v);
+  a.codes = codes;
+  a.scales = scales;
+  a.N = (int)N;
+  a.B = (int)q->B;
+  a.Hr = (int)(q->H / N);
+  a.Hc = (int)hc;
+  a.h0 = (int)h0;
+  a.Lr = (int)q->L;
+  a.rows = (long long)N * q->B * hc * q->L * 3;
+  return launch_ulysses<lx::kPackQKV>(a, q->D, stream);
+}
+
+lx_status lx_ulysses_unpack_qkv(const uint8_t* codes, const float* scales, int64_t N, const lx_bhld* q,
+                                const lx_bhld* k, const lx_bhld* v, cudaStream_t stream) {
+  lx_status st;
+  if ((st = check_bhld(q)) != LX_OK || (st = check_bhld(k)) != LX_OK || (st = check_bhld(v)) != LX_OK) return st;
+  if (!same_shape(q, k) || !same_shape(q, v) || !codes || !scales) return LX_ERR_INVALID;
+  if (N < 1 || q->L % N != 0) return LX_ERR_INVALID;
+  if (!al16(codes) || !al16(scales)) return LX_ERR_ALIGN;
+  lx::UlyssesArgs a{};
+  a.x[0] = rw(q);
+  a.x[1] = rw(k);
+  a.x[2] = rw(v);
+  a.codes = const_cast<uint8_t*>(codes);
+  a.scales = const_cast<float*>(scales);
+  a.N = (int)N;
+  a.B = (int)q->B;
+  a.Hr = (int)q->H;
+  a.Hc = (int)q->H;
+  a.Lr = (int)(q->L / N);
+  a.rows = (long long)N * q->B * q->H * (q->L / N) * 3;
+  return launch_ulysses<lx::kUnpackQKV>(a, q->D, stream);
+}
+
+lx_status lx_ulysses_pack_o(const lx_bhld* o, int64_t N, uint8_t* codes, float* scales, cudaStream_t stream) {
+  lx_status st;
+  if ((st = check_bhld(o)) != LX_OK) return st;
+  if (!codes || !scales || N < 1 || o->L % N != 0) return LX_ERR_INVALID;
+  if (!al16(codes) || !al16(scales)) return LX_ERR_ALIGN;
+  lx::UlyssesArgs a{};
+  a.x[0] = rw(o);
+  a.codes = codes;
+  a.scales = scales;
+  a.N = (int)N;
+  a.B = (int)o->B;
+  a.Hr = (int)o->H;
+  a.Hc = (int)o->H;
+  a.Lr = (int)(o->L / N);
+  a.rows = (long long)N * o->B * o->H * (o->L / N);
+  return launch_ulysses<lx::kPackO>(a, o->D, stream);
+}
+
+lx_status lx_ulysses_unpack_o(const uint8_t* codes, const float* scales, int64_t N, int64_t h0, int64_t hc,
+                              const lx_bhld* out, cudaStream_t stream) {
+  lx_status st;
+  if ((st = check_bhld(out)) != LX_OK) return st;
+  if (!codes || !scales || N < 1 || out->H % N != 0 || h0 < 0 || hc < 1 || h0 + hc > out->H / N)
+    return LX_ERR_INVALID;
+  if (!al16(codes) || !al16(scales)) return LX_ERR_ALIGN;
+  lx::UlyssesArgs a{};
+  a.x[0] = rw(out);
+  a.codes = const_cast<uint8_t*>(codes);
+  a.scales = const_cast<float*>(scales);
+  a.N = (int)N;
+  a.B = (int)out->B;
+  a.Hr = (int)(out->H / N);
+  a.Hc = (int)hc;
+  a.h0 = (int)h0;
+  a.Lr = (int)out->L;
+  a.rows = (long long)N * out->B * hc * out->L;
+  return launch_ulysses<lx::kUnpackO>(a, out->D, stream);
 }
 
 }  // extern "C"
