@@ -42,7 +42,7 @@ def _worker(rank, world, port, out):
 @pytest.mark.parametrize("world", [2, 4])
 def test_max_over_ranks_and_job_value(world):
     port = _free_port()
-    with mp.Manager() as m:
+    with mp.get_context("spawn").Manager() as m:
         out = m.dict()
         mp.start_processes(_worker, args=(world, port, out), nprocs=world, start_method="spawn", join=True)
         res = dict(out)

@@ -81,7 +81,7 @@ def _worker(rank, world, port, n_chunks, out):
 def test_exchange_round_trip_across_ranks(world, n_chunks):
     import oracle
     port = _free_port()
-    with mp.Manager() as m:
+    with mp.get_context("spawn").Manager() as m:
         out = m.dict()
         mp.start_processes(_worker, args=(world, port, n_chunks, out), nprocs=world, start_method="spawn", join=True)
         res = dict(out)
