@@ -329,6 +329,89 @@ def run_ours(args, rank, world, local_rank):
     return out
 
 
+# ------------------------------------------------------------------ Light-Ulysses share
+def run_ulysses_share(args):
+    """One rank's share of an N-GPU Light-Ulysses step at the workload's grid,
+    timed on one GPU: pack this rank's token shard (all heads) into the FP8
+    payload, unpack a payload of the same layout (the send buffer stands in for
+    the received one: with one GPU there is no exchange), the attention of the
+    H/N heads over all tokens, then the output's pack and unpack.  Reports each
+    exchange kernel against the HBM roofline; the all-to-all itself is not
+    timed."""
+    import torch
+
+    import video_dit_dynamic_token_b200 as lx
+    from video_dit_dynamic_token_b200 import synth, ulysses
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    w = synth.WORKLOADS[args.workload]
+    N = args.ulysses
+    B, H, d, L = w.B, w.H, w.d, w.L
+    if H % N or L % N:
+        raise SystemExit("heads and tokens must divide by N")
+    Hr, Lr = H // N, L // N
+    keep = args.keep if args.keep else w.keep
+    g = torch.Generator(device=dev).manual_seed(0)
+    q, k, v = ((torch.randn(B, Lr, H, d, generator=g, device=dev)).to(torch.bfloat16) for _ in range(3))
+    qv, kv, vv = (x.permute(0, 2, 1, 3) for x in (q, k, v))
+    c = torch.empty((N, B, Hr, Lr, 3, d), dtype=torch.uint8, device=dev)
+    sc = torch.empty((N, B, Hr, Lr, 3), dtype=torch.float32, device=dev)
+    qh, kh, vh = (torch.empty((B, Hr, L, d), dtype=torch.bfloat16, device=dev) for _ in range(3))
+    oc = torch.empty((N, B, Hr, Lr, d), dtype=torch.uint8, device=dev)
+    osc = torch.empty((N, B, Hr, Lr), dtype=torch.float32, device=dev)
+    out = torch.empty_like(q)
+    ws = torch.empty(lx.lx_sparse_attn_ws_size(qh, keep, args.mode), dtype=torch.uint8, device=dev)
+    oh = torch.empty_like(qh)
+    names = ["pack_qkv", "unpack_qkv", "attn", "pack_o", "unpack_o"]
+
+    def step(ev=None):
+        def mark(i):
+            if ev is not None:
+                ev[i].record()
+        mark(0)
+        ulysses.pack_qkv(qv, kv, vv, N, 0, Hr, c, sc)
+        mark(1)
+        ulysses.unpack_qkv(c, sc, N, qh, kh, vh)
+        mark(2)
+        lx.lx_sparse_attn(qh, kh, vh, keep, args.mode, out=oh, ws=ws)
+        mark(3)
+        ulysses.pack_o(oh, N, oc, osc)
+        mark(4)
+        ulysses.unpack_o(oc, osc, N, 0, Hr, out.permute(0, 2, 1, 3))
+        mark(5)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(args.steps)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record()
+    for i in range(args.steps):
+        step(evs[i])
+    t1.record()
+    torch.cuda.synchronize()
+    if lx.lx_last_device_status() != 0:
+        raise RuntimeError("device status error")
+    ms = t0.elapsed_time(t1) / args.steps
+    per = {n: sum(e[j].elapsed_time(e[j + 1]) for e in evs) / args.steps for j, n in enumerate(names)}
+    peaks = _peaks()
+    rows_qkv, rows_o = 3 * B * H * Lr, B * H * Lr     # one rank's payload rows (all destinations)
+    byt = {"pack_qkv": rows_qkv * (2 * d + d + 4), "unpack_qkv": rows_qkv * (d + 4 + 2 * d),
+           "pack_o": rows_o * (2 * d + d + 4), "unpack_o": rows_o * (d + 4 + 2 * d)}
+    phases = {n: {"ms": round(per[n], 4), "algorithmic_mb": round(b / 1e6, 1),
+                  "gbs": round(b / (per[n] * 1e-3) / 1e9, 1),
+                  "hbm_frac": round(b / (per[n] * 1e-3) / 1e9 / peaks["hbm_gbs"], 3)} for n, b in byt.items()}
+    flops = lx.effective_flops(B, Hr, L, d, keep)
+    return {"metric": f"Light-Ulysses one-rank share of an N={N} step ({args.workload} grid, {H}x{d}, keep {keep})",
+            "value": round(flops / (ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s", "n_gpus": 1, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(ms, 4), "higher_is_better": True, "dtype": args.mode,
+            "data": "synthetic N(0,1) shards", "config": {"workload": f"{args.workload} B={B} H={H} d={d} L={L} N={N}",
+                                                          "shard_tokens": Lr, "heads_after_exchange": Hr},
+            "breakdown_ms": {n: round(v, 4) for n, v in per.items()}, "phases": phases,
+            "note": "the all-to-all is not timed (one GPU); the send buffer stands in for the received one"}
+
+
 # ------------------------------------------------------------------ CPU oracle timing
 def cpu_oracle_sample(seconds_target=12.0):
     """Time the oracle (as it stands) on one head of the workload: planner and
@@ -408,9 +491,14 @@ def main():
     ap.add_argument("--keep", type=float, default=0.0, help="override the workload's keep ratio (sweeps)")
     ap.add_argument("--smooth-k", action="store_true",
                     help="int8fp8: K smoothing (channel means of K subtracted before its INT8 codes)")
+    ap.add_argument("--ulysses", type=int, default=0,
+                    help="time one rank's share of an N-GPU Light-Ulysses step instead (exchange kernels + attention)")
     ap.add_argument("--prologue", action="store_true",
                     help="int8fp8: the Q/K pass also applies per-head RMSNorm and 3D RoPE (lx_qk_prologue)")
     args = ap.parse_args()
+    if args.ulysses:
+        print(json.dumps(run_ulysses_share(args)))
+        return
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))

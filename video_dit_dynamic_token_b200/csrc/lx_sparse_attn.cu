@@ -274,12 +274,16 @@ lx::BhldRW rw(const lx_bhld* t) {
 template <int MODE>
 lx_status launch_ulysses(lx::UlyssesArgs a, int64_t D, cudaStream_t s) {
   if (a.rows == 0) return LX_OK;
-  const long long threads = a.rows * (D / 8);
-  const unsigned blocks = (unsigned)((threads + 255) / 256);
+  // blockIdx.y: the (destination, batch, head) slices; blockIdx.x: rows of one slice
+  const long long slices = (long long)a.N * a.B * a.Hc;
+  const long long slice_rows = (long long)a.Lr * ((MODE == lx::kPackQKV || MODE == lx::kUnpackQKV) ? 3 : 1);
+  const long long per_block = (256 / (D / 8)) * (long long)lx::kUlyPasses;  // rows per CTA
+  if (slices > 65535 || slice_rows > (1LL << 30)) return LX_ERR_UNSUPPORTED;
+  dim3 grid((unsigned)((slice_rows + per_block - 1) / per_block), (unsigned)slices);
   if (D == 128)
-    lx::ulysses_rows_kernel<128, MODE><<<blocks, 256, 0, s>>>(a);
+    lx::ulysses_rows_kernel<128, MODE><<<grid, 256, 0, s>>>(a);
   else
-    lx::ulysses_rows_kernel<64, MODE><<<blocks, 256, 0, s>>>(a);
+    lx::ulysses_rows_kernel<64, MODE><<<grid, 256, 0, s>>>(a);
   return launch_status();
 }
 }  // namespace

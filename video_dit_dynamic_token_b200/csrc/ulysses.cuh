@@ -52,73 +52,93 @@ __device__ __forceinline__ void e4m3x4_to_f32(uint32_t c, float (&f)[4]) {
 }
 
 // One payload row per D/8 consecutive lanes (16 bytes of bf16 or 8 bytes of
-// codes each), in payload order.
+// codes each).  blockIdx.y is the (destination n, batch b, head j) slice of the
+// payload, decoded once per CTA; blockIdx.x walks the slice's Lr*X rows (X = 3
+// for the Q/K/V payload: row = 3 t + tensor), kUlyPasses groups per lane group,
+// with every pass's loads issued before any of them is used.
+constexpr int kUlyPasses = 4;
+
 template <int D, int MODE>
 __global__ void __launch_bounds__(256) ulysses_rows_kernel(UlyssesArgs a) {
   constexpr int CH = D / 8;
-  const long long row = ((long long)blockIdx.x * blockDim.x + threadIdx.x) / CH;
-  const int c = threadIdx.x % CH;
-  const bool live = row < a.rows;
-  const long long rr = live ? row : 0;
-  // payload coordinates of the row
+  constexpr int G = 256 / CH;  // row groups per pass
   constexpr bool QKV = MODE == kPackQKV || MODE == kUnpackQKV;
-  long long q = rr;
-  int x = 0;
-  if (QKV) {
-    x = (int)(q % 3);
-    q /= 3;
+  constexpr int X = QKV ? 3 : 1;
+  const int c = threadIdx.x % CH, g = threadIdx.x / CH;
+  const int ny = blockIdx.y;
+  const int j = ny % a.Hc;
+  const int b = (ny / a.Hc) % a.B;
+  const int n = ny / (a.Hc * a.B);
+  const int slice_rows = a.Lr * X;
+  const long long slice0 = (long long)ny * slice_rows;  // payload row of the slice's first row
+  const int base = blockIdx.x * G * kUlyPasses;
+  __nv_bfloat16* xr[kUlyPasses];
+  long long pr[kUlyPasses];
+  bool live[kUlyPasses];
+#pragma unroll
+  for (int i = 0; i < kUlyPasses; ++i) {
+    const int lr = base + i * G + g;
+    live[i] = lr < slice_rows;
+    const int l = live[i] ? lr : 0;
+    const int x = QKV ? l % 3 : 0;
+    const int t = QKV ? l / 3 : l;
+    const BhldRW& T = a.x[x];
+    long long head, tok;
+    if (MODE == kPackQKV || MODE == kUnpackO) {  // sequence shard, all heads
+      head = (long long)n * a.Hr + a.h0 + j;
+      tok = t;
+    } else {                                      // head chunk, all tokens
+      head = j;
+      tok = (long long)n * a.Lr + t;
+    }
+    xr[i] = T.p + b * T.sB + head * T.sH + tok * T.sL + c * 8;
+    pr[i] = slice0 + l;
   }
-  const int t = (int)(q % a.Lr);
-  q /= a.Lr;
-  const int j = (int)(q % a.Hc);
-  q /= a.Hc;
-  const int b = (int)(q % a.B);
-  const int n = (int)(q / a.B);
-  // the bf16 row this payload row comes from or goes to
-  const BhldRW& X = a.x[QKV ? x : 0];
-  long long head, tok;
-  if (MODE == kPackQKV || MODE == kUnpackO) {  // sequence shard, all heads
-    head = (long long)n * a.Hr + a.h0 + j;
-    tok = t;
-  } else {                                      // head chunk, all tokens
-    head = j;
-    tok = (long long)n * a.Lr + t;
-  }
-  __nv_bfloat16* xrow = X.p + b * X.sB + head * X.sH + tok * X.sL + c * 8;
-  uint8_t* crow = a.codes + rr * D + c * 8;
   if constexpr (MODE == kPackQKV || MODE == kPackO) {
-    const uint4 v = live ? ld_stream_v4(xrow) : make_uint4(0, 0, 0, 0);
-    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-    float m = 0.f;
+    uint4 v[kUlyPasses];
 #pragma unroll
-    for (int e = 0; e < 4; ++e) m = fmaxf(m, fmaxf(fabsf(bf16lo(w[e])), fabsf(bf16hi(w[e]))));
+    for (int i = 0; i < kUlyPasses; ++i) v[i] = live[i] ? ld_stream_v4(xr[i]) : make_uint4(0, 0, 0, 0);
 #pragma unroll
-    for (int off = 1; off < CH; off <<= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
-    const float inv = m > 0.f ? __fdiv_rn(448.0f, m) : 0.f;
-    const uint32_t c0 = e4m3x4(__fmul_rn(bf16lo(w[0]), inv), __fmul_rn(bf16hi(w[0]), inv),
-                               __fmul_rn(bf16lo(w[1]), inv), __fmul_rn(bf16hi(w[1]), inv));
-    const uint32_t c1 = e4m3x4(__fmul_rn(bf16lo(w[2]), inv), __fmul_rn(bf16hi(w[2]), inv),
-                               __fmul_rn(bf16lo(w[3]), inv), __fmul_rn(bf16hi(w[3]), inv));
-    if (live) {
-      *reinterpret_cast<uint2*>(crow) = make_uint2(c0, c1);
-      if (c == 0) a.scales[rr] = m > 0.f ? __fdiv_rn(m, 448.0f) : 1.0f;
+    for (int i = 0; i < kUlyPasses; ++i) {
+      const uint32_t w[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
+      float m = 0.f;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) m = fmaxf(m, fmaxf(fabsf(bf16lo(w[e])), fabsf(bf16hi(w[e]))));
+#pragma unroll
+      for (int off = 1; off < CH; off <<= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+      const float inv = m > 0.f ? __fdiv_rn(448.0f, m) : 0.f;
+      const uint32_t c0 = e4m3x4(__fmul_rn(bf16lo(w[0]), inv), __fmul_rn(bf16hi(w[0]), inv),
+                                 __fmul_rn(bf16lo(w[1]), inv), __fmul_rn(bf16hi(w[1]), inv));
+      const uint32_t c1 = e4m3x4(__fmul_rn(bf16lo(w[2]), inv), __fmul_rn(bf16hi(w[2]), inv),
+                                 __fmul_rn(bf16lo(w[3]), inv), __fmul_rn(bf16hi(w[3]), inv));
+      if (live[i]) {
+        *reinterpret_cast<uint2*>(a.codes + pr[i] * D + c * 8) = make_uint2(c0, c1);
+        if (c == 0) a.scales[pr[i]] = m > 0.f ? __fdiv_rn(m, 448.0f) : 1.0f;
+      }
     }
   } else {
-    if (live) {
-      const uint2 cw = *reinterpret_cast<const uint2*>(crow);
-      const float s = a.scales[rr];
+    uint2 cw[kUlyPasses];
+    float s[kUlyPasses];
+#pragma unroll
+    for (int i = 0; i < kUlyPasses; ++i) {
+      cw[i] = live[i] ? *reinterpret_cast<const uint2*>(a.codes + pr[i] * D + c * 8) : make_uint2(0, 0);
+      s[i] = live[i] ? a.scales[pr[i]] : 0.f;
+    }
+#pragma unroll
+    for (int i = 0; i < kUlyPasses; ++i) {
+      if (!live[i]) continue;
       float f0[4], f1[4];
-      e4m3x4_to_f32(cw.x, f0);
-      e4m3x4_to_f32(cw.y, f1);
+      e4m3x4_to_f32(cw[i].x, f0);
+      e4m3x4_to_f32(cw[i].y, f1);
       uint32_t o[4];
 #pragma unroll
       for (int e = 0; e < 2; ++e) {
-        __nv_bfloat162 p0 = __floats2bfloat162_rn(__fmul_rn(f0[2 * e], s), __fmul_rn(f0[2 * e + 1], s));
-        __nv_bfloat162 p1 = __floats2bfloat162_rn(__fmul_rn(f1[2 * e], s), __fmul_rn(f1[2 * e + 1], s));
+        __nv_bfloat162 p0 = __floats2bfloat162_rn(__fmul_rn(f0[2 * e], s[i]), __fmul_rn(f0[2 * e + 1], s[i]));
+        __nv_bfloat162 p1 = __floats2bfloat162_rn(__fmul_rn(f1[2 * e], s[i]), __fmul_rn(f1[2 * e + 1], s[i]));
         o[e] = *reinterpret_cast<uint32_t*>(&p0);
         o[2 + e] = *reinterpret_cast<uint32_t*>(&p1);
       }
-      *reinterpret_cast<uint4*>(xrow) = make_uint4(o[0], o[1], o[2], o[3]);
+      *reinterpret_cast<uint4*>(xr[i]) = make_uint4(o[0], o[1], o[2], o[3]);
     }
   }
 }
