@@ -5,6 +5,14 @@ Thin Python binding over the C-ABI library ``liblx_sparse_attn.so`` (see
 arguments: torch allocates device memory and supplies the current stream, and
 every step of the computation runs in the library's CUDA kernels.  There is no
 CPU fallback -- a missing library raises.
+
+Entry points: the planner (lx_pool_means, lx_score_topk, lx_sparse_attn_plan),
+the quantisers (lx_quantize_qk, lx_pool_quantize_qk, lx_quantize_v), the
+attention (lx_attn_bf16, lx_attn_int8fp8, lx_sparse_attn_fwd), plan and
+forward in one call (lx_sparse_attn), the fused Q/K prologue (lx_rope3d_table,
+lx_qk_prologue), K smoothing (lx_k_channel_mean, lx_quantize_qk_smooth,
+lx_pool_quantize_qk_smooth); the host-to-host pipeline is in ``pipeline`` and
+the Light-Ulysses exchange in ``ulysses``.
 """
 from __future__ import annotations
 
@@ -194,31 +202,23 @@ def lx_qk_prologue(Q, K, wq, wk, eps, grid, theta=10000.0, split=None, table=Non
                    stream=None):
     """Per-head RMSNorm + 3D RoPE of Q and K, with the block means and INT8 codes
     of the bf16 result, in one pass: dict(Yq, Yk, mq, mk, qc, qs, kc, ks)."""
-    lib = _abi.load()
     B, H, L, D = Q.shape
     nB = (L + LX_BLOCK - 1) // LX_BLOCK
     dev = Q.device
     if table is None:
         table = lx_rope3d_table(grid, D, theta, split, dev, stream)
-    r = _rope(grid, D, theta, split)
     out = {"mq": torch.empty((B, H, nB, D), dtype=torch.float32, device=dev),
            "mk": torch.empty((B, H, nB, D), dtype=torch.float32, device=dev)}
-    yq = yk = None
     if with_y:
         out["Yq"] = torch.empty((B, H, L, D), dtype=torch.bfloat16, device=dev)
         out["Yk"] = torch.empty((B, H, L, D), dtype=torch.bfloat16, device=dev)
-        yq, yk = bhld(out["Yq"]), bhld(out["Yk"])
     if with_codes:
         out["qc"] = torch.empty((B, H, L, D), dtype=torch.int8, device=dev)
         out["qs"] = torch.empty((B, H, nB), dtype=torch.float32, device=dev)
         out["kc"] = torch.empty((B, H, L, D), dtype=torch.int8, device=dev)
         out["ks"] = torch.empty((B, H, nB), dtype=torch.float32, device=dev)
-    q, k = bhld(Q), bhld(K)
-    p = lambda name: _ptr(out[name]) if name in out else None
-    _check(lib.lx_qk_prologue(ctypes.byref(q), ctypes.byref(k), _ptr(wq), _ptr(wk), float(eps), ctypes.byref(r),
-                              _ptr(table), ctypes.byref(yq) if yq is not None else None,
-                              ctypes.byref(yk) if yk is not None else None, p("mq"), p("mk"), p("qc"), p("qs"),
-                              p("kc"), p("ks"), _stream(stream)), "lx_qk_prologue")
+    lx_qk_prologue_into(Q, K, wq, wk, eps, grid, table, out["mq"], out["mk"], out.get("qc"), out.get("qs"),
+                        out.get("kc"), out.get("ks"), out.get("Yq"), out.get("Yk"), theta, split, stream)
     return out
 
 
