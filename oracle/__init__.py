@@ -13,3 +13,6 @@ from .prologue_ref import (ROPE_THETA, bf16_round, k_channel_mean_ref, prologue_
                            qk_rmsnorm_ref, quant_k_smooth_ref, rope3d_ref, rope3d_split, token_positions)
 from .ulysses_ref import (all_to_all_ref, fp8_rows_dequant_ref, fp8_rows_ref, pack_o_ref, pack_qkv_ref,  # noqa: F401
                           unpack_o_ref, unpack_qkv_ref)
+from .nvfp4_ref import (E2M1_MAX, NVFP4_BLOCK, dequant_nvfp4_ref, e2m1_decode, e2m1_encode,  # noqa: F401
+                         e2m1_round, gemm_nvfp4_ref, nvfp4_global_scale, pack_e2m1, quant_nvfp4_ref, sf_tiled,
+                         unpack_e2m1)
