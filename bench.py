@@ -412,6 +412,111 @@ def run_ulysses_share(args):
             "note": "the all-to-all is not timed (one GPU); the send buffer stands in for the received one"}
 
 
+# ------------------------------------------------------------------ NVFP4 linear
+GEMM_WORKLOAD = "Wan2.2-A14B fused QKV projection, 720p grid: M=75600 tokens, K=5120, N=15360, fp32 bias"
+
+
+def nvfp4_cpu_sample(M, N, K, rows=32):
+    """The oracle (quantisation + fp64 GEMM) on `rows` rows of the workload."""
+    import numpy as np
+
+    import oracle
+    rng = np.random.default_rng(0)
+    t0 = time.perf_counter()
+    X = rng.standard_normal((rows, K)).astype(np.float32)
+    W = (rng.standard_normal((N, K)) * 0.02).astype(np.float32)
+    t1 = time.perf_counter()
+    xq = oracle.quant_nvfp4_ref(X)
+    wq = oracle.quant_nvfp4_ref(W)
+    oracle.gemm_nvfp4_ref(xq, wq, np.zeros(N, np.float32))
+    dt = time.perf_counter() - t1
+    flops = 2.0 * rows * N * K
+    return {"value": round(flops / dt / 1e12, 6), "unit": "TFLOP/s", "cores": os.cpu_count(), "kind": "oracle",
+            "sample": f"{rows} of the {M} rows (weights quantised in the sample too), {dt:.1f} s",
+            "setup_s": round(t1 - t0, 1)}
+
+
+def run_nvfp4_gemm(args):
+    """One step = one NVFP4 linear layer: quantise the bf16 activations (amax
+    pass, global scale, quantiser) and run the block-scaled GEMM with the column
+    bias; the weights are quantised once, before timing, as a deployed model's
+    would be.  X (774 MB) is larger than L2, so no flush is needed."""
+    import torch
+
+    import video_dit_dynamic_token_b200 as lx
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    M, N, K = (args.gemm_m or 75600), 15360, 5120
+    g = torch.Generator(device=dev).manual_seed(0)
+    X = torch.randn((M, K), generator=g, device=dev).to(torch.bfloat16)
+    W = (torch.randn((N, K), generator=g, device=dev) * 0.02).to(torch.bfloat16)
+    bias = torch.randn(N, generator=g, device=dev) * 0.1
+    wq = lx.lx_nvfp4_quantize(W)
+    xq = lx.lx_nvfp4_quantize(X)
+    Y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        lx.lx_nvfp4_quantize(X, out=xq)
+        if ev is not None:
+            ev[1].record(stream)
+        lx.lx_nvfp4_gemm(xq, wq, bias, out=Y)
+        if ev is not None:
+            ev[2].record(stream)
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize()
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(0)
+    clocks.start()
+    torch.cuda.synchronize()
+    t0.record(stream)
+    for i in range(args.steps):
+        step(evs[i])
+    t1.record(stream)
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    if lx.lx_last_device_status() != 0:
+        raise RuntimeError("device status error")
+    ms = t0.elapsed_time(t1) / args.steps
+    q_ms = sum(e[0].elapsed_time(e[1]) for e in evs) / args.steps
+    g_ms = sum(e[1].elapsed_time(e[2]) for e in evs) / args.steps
+    flops = lx.nvfp4_gemm_flops(M, N, K)
+    peaks = _peaks()
+    fp4_peak = 4.0 * peaks["bf16"]   # dense fp4 : bf16 = 9 : 2.25 PFLOP/s nominal
+    q_bytes = 2 * (M * K * 2) + M * K // 2 + M * K // 16   # two reads of X (amax, quantiser), codes + scales
+    g_bytes = M * K // 2 + M * K // 16 + N * K // 2 + N * K // 16 + M * N * 2 + N * 4
+    out = {"metric": "NVFP4 linear (activation quantisation + block-scaled GEMM + bias) TFLOP/s",
+           "value": round(flops / (ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s", "n_gpus": 1, "steps": args.steps,
+           "warmup": max(3, args.warmup), "ms_per_step": round(ms, 4), "higher_is_better": True, "scaling": "weak",
+           "vs_baseline": None, "dtype": "nvfp4 (e2m1 x e2m1, e4m3/16 scales, f32 accumulate, bf16 out)",
+           "data": "synthetic: X ~ N(0,1), W ~ N(0, 0.02^2), bias ~ N(0, 0.01)",
+           "config": {"workload": GEMM_WORKLOAD if M == 75600 else f"NVFP4 QKV projection, M={M}, K={K}, N={N}",
+                      "M": M, "N": N, "K": K, "l2": "inputs larger than L2 (X 774 MB)"},
+           "breakdown_ms": {"quantise_x": round(q_ms, 4), "gemm": round(g_ms, 4)},
+           "roofline": {"bound": "tensor", "achieved": round(flops / (g_ms * 1e-3) / 1e12, 1),
+                        "peak": round(fp4_peak, 1), "unit": "TFLOP/s",
+                        "frac": round(flops / (g_ms * 1e-3) / 1e12 / fp4_peak, 3), "traffic": None,
+                        "peak_source": f"{peaks['source']} bf16 burst x 4 (nominal dense fp4/bf16 ratio)",
+                        "kernel": "nvfp4_gemm_kernel"},
+           "phases": {"quantise_x": {"ms": round(q_ms, 4), "algorithmic_mb": round(q_bytes / 1e6, 1),
+                                     "gbs": round(q_bytes / (q_ms * 1e-3) / 1e9, 1),
+                                     "hbm_frac": round(q_bytes / (q_ms * 1e-3) / 1e9 / peaks["hbm_gbs"], 3)},
+                      "gemm": {"ms": round(g_ms, 4), "algorithmic_mb": round(g_bytes / 1e6, 1),
+                               "hbm_frac_of_time": round(g_bytes / (g_ms * 1e-3) / 1e9 / peaks["hbm_gbs"], 3)}},
+           "gpu_launches": 4 * args.steps, "clocks": clk, "e2e": None,
+           "note": "sub-benchmark of the NVFP4 projection kernel; the headline line (no flags) carries e2e"}
+    if not args.no_cpu_baseline:
+        out["cpu_baseline"] = nvfp4_cpu_sample(M, N, K)
+    if M != 75600:
+        out["note"] = "smaller M: a profiling case, not the benchmark"
+    return out
+
 # ------------------------------------------------------------------ CPU oracle timing
 def cpu_oracle_sample(seconds_target=12.0):
     """Time the oracle (as it stands) on one head of the workload: planner and
@@ -495,7 +600,13 @@ def main():
                     help="time one rank's share of an N-GPU Light-Ulysses step instead (exchange kernels + attention)")
     ap.add_argument("--prologue", action="store_true",
                     help="int8fp8: the Q/K pass also applies per-head RMSNorm and 3D RoPE (lx_qk_prologue)")
+    ap.add_argument("--gemm", action="store_true",
+                    help="time one NVFP4 linear layer (the 720p fused QKV projection) instead")
+    ap.add_argument("--gemm-m", type=int, default=0, help="--gemm with fewer token rows: a profiling case only")
     args = ap.parse_args()
+    if args.gemm:
+        print(json.dumps(run_nvfp4_gemm(args)))
+        return
     if args.ulysses:
         print(json.dumps(run_ulysses_share(args)))
         return

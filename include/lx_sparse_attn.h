@@ -282,6 +282,49 @@ lx_status lx_sparse_attn_ws_size(const lx_bhld* Q, double keep, lx_mode mode, si
 lx_status lx_sparse_attn(const lx_bhld* Q, const lx_bhld* K, const lx_bhld* V, double keep, lx_mode mode,
                          lx_plan* plan, const lx_bhld* O, void* ws, size_t ws_bytes, cudaStream_t stream);
 
+/* ---------------------------------------------------------------- NVFP4
+ * "Run Wan2.2-A14B on One RTX 5090: 720p Video in 3.8s", §2 (NVFP4
+ * quantization-aware training): NVFP4 = E2M1 values, one E4M3 scale per 16
+ * consecutive elements, one FP32 scale per tensor; the linear layers run a
+ * block-scaled GEMM of NVFP4 activations by NVFP4 weights with FP32
+ * accumulation, BF16 output and the column bias fused in the epilogue.
+ *
+ * Scale rule (this library's reading; the pages give only the format), in fp32:
+ *   g   = amax / 2688 (1 for an all-zero tensor),  ig6 = 1 / (6 g)
+ *   s   = E4M3_rn_satfinite(amax_block * ig6),  inv = 1 / (s g)  (0 when s = 0)
+ *   code = E2M1_rn_satfinite(x * inv) (ties to even; a zero result is +0)
+ * each product and reciprocal rounded to fp32 once.
+ *
+ * Layouts (device memory, dense):
+ *   codes  uint8 [R][K/2]: element 2i in the low nibble of byte i of the row;
+ *   scales uint8, tiled for the tensor core: rows padded to a multiple of 128
+ *          (padding scales are 0); the E4M3 scale of row r, 16-element block j
+ *          sits at byte (t*KS + ks)*512 + l*16 + c*4 + jj with t = r/128,
+ *          l = r%32, c = (r%128)/32, ks = j/4, jj = j%4, KS = K/64.
+ *   global scale: one fp32 in device memory. */
+
+/* Bytes of the code and scale buffers of an [R, K] tensor (K % 64 == 0). */
+lx_status lx_nvfp4_sizes(int64_t R, int64_t K, size_t* code_bytes, size_t* sf_bytes);
+
+/* Quantise bf16 x [R, K] (row stride ldx elements, ldx % 8 == 0, K % 64 == 0,
+ * 16-byte aligned) to NVFP4.  compute_gscale != 0: *gscale (device fp32) is
+ * computed from x and written (an amax pass, then the quantiser); 0: *gscale
+ * is read as given.  codes / sf: buffers of lx_nvfp4_sizes bytes, 16-byte
+ * aligned, owned by the caller.  Finite inputs only. */
+lx_status lx_nvfp4_quantize(const void* x, int64_t R, int64_t K, int64_t ldx, int compute_gscale, float* gscale,
+                            uint8_t* codes, uint8_t* sf, cudaStream_t stream);
+
+/* Y[m, n] = bf16(fl32(acc[m, n] * fl32(gx * gw)) + bias[n]), acc = the fp32
+ * tensor-core sum over k of x[m, k] w[n, k] (each the E2M1 value times its E4M3
+ * block scale): X = (xc, xsf, gx) [M, K], W = (wc, wsf, gw) [N, K] as written by
+ * lx_nvfp4_quantize; bias fp32 [N] or NULL; y bf16 [M, N] with row stride ldy
+ * (ldy % 8 == 0, 16-byte aligned).  N % 128 == 0, K % 256 == 0; M is any
+ * count >= 1 up to 65535*128.  A wait that runs out sets the device status
+ * to LX_ERR_TIMEOUT (see lx_last_device_status). */
+lx_status lx_nvfp4_gemm(const uint8_t* xc, const uint8_t* xsf, const float* gx, const uint8_t* wc,
+                        const uint8_t* wsf, const float* gw, const float* bias, int64_t M, int64_t N, int64_t K,
+                        void* y, int64_t ldy, cudaStream_t stream);
+
 /* Synchronises `stream`, returns and clears the device status word of the
  * current device: LX_OK, LX_ERR_TIMEOUT, LX_ERR_PLAN, or LX_ERR_CUDA when the
  * stream itself reports an error. */

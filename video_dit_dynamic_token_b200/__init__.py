@@ -11,8 +11,9 @@ the quantisers (lx_quantize_qk, lx_pool_quantize_qk, lx_quantize_v), the
 attention (lx_attn_bf16, lx_attn_int8fp8, lx_sparse_attn_fwd), plan and
 forward in one call (lx_sparse_attn), the fused Q/K prologue (lx_rope3d_table,
 lx_qk_prologue), K smoothing (lx_k_channel_mean, lx_quantize_qk_smooth,
-lx_pool_quantize_qk_smooth); the host-to-host pipeline is in ``pipeline`` and
-the Light-Ulysses exchange in ``ulysses``.
+lx_pool_quantize_qk_smooth), NVFP4 (lx_nvfp4_quantize, lx_nvfp4_gemm); the
+host-to-host pipeline is in ``pipeline`` and the Light-Ulysses exchange in
+``ulysses``.
 """
 from __future__ import annotations
 
@@ -375,6 +376,63 @@ def lx_sparse_attn(Q, K, V, keep, mode="int8fp8", plan: Plan | None = None, out=
                               ctypes.byref(cp), ctypes.byref(o), _ptr(ws), ws.numel(), _stream(stream)),
            "lx_sparse_attn")
     return out, plan
+
+
+
+# ---------------------------------------------------------------- NVFP4
+@dataclass
+class NvFp4Tensor:
+    """An NVFP4 tensor [R, K] in the layouts of lx_nvfp4_quantize: codes uint8
+    [R, K/2], tiled E4M3 scales (uint8, rows padded to 128), fp32 global scale [1]."""
+    codes: torch.Tensor
+    sf: torch.Tensor
+    gscale: torch.Tensor
+    R: int
+    K: int
+
+
+def lx_nvfp4_sizes(R, K):
+    cb, sb = ctypes.c_size_t(), ctypes.c_size_t()
+    _check(_abi.load().lx_nvfp4_sizes(int(R), int(K), ctypes.byref(cb), ctypes.byref(sb)), "lx_nvfp4_sizes")
+    return cb.value, sb.value
+
+
+def lx_nvfp4_quantize(x, gscale=None, out: NvFp4Tensor | None = None, stream=None) -> NvFp4Tensor:
+    """x: bf16 [R, K] CUDA tensor with contiguous rows.  gscale None: the global
+    scale is computed from x; else a CUDA fp32 tensor of one element used as given."""
+    if x.dtype != torch.bfloat16 or x.dim() != 2 or x.stride(1) != 1:
+        raise ValueError("expected a bf16 [R, K] tensor with contiguous rows")
+    R, K = x.shape
+    if out is None:
+        cb, sb = lx_nvfp4_sizes(R, K)
+        g = torch.empty(1, dtype=torch.float32, device=x.device)
+        out = NvFp4Tensor(torch.empty((R, K // 2), dtype=torch.uint8, device=x.device),
+                          torch.empty(sb, dtype=torch.uint8, device=x.device), g, R, K)
+    compute = gscale is None
+    if not compute:
+        out.gscale.copy_(gscale.reshape(1))
+    _check(_abi.load().lx_nvfp4_quantize(_ptr(x), R, K, x.stride(0), int(compute), _ptr(out.gscale), _ptr(out.codes),
+                                         _ptr(out.sf), _stream(stream)), "lx_nvfp4_quantize")
+    return out
+
+
+def lx_nvfp4_gemm(xq: NvFp4Tensor, wq: NvFp4Tensor, bias=None, out=None, stream=None):
+    """Y = X W^T + bias in bf16 [M, N] from NVFP4 X [M, K] and W [N, K]; bias fp32 [N] or None."""
+    if xq.K != wq.K:
+        raise ValueError("X and W differ in K")
+    M, N, K = xq.R, wq.R, xq.K
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.bfloat16, device=xq.codes.device)
+    if bias is not None and (bias.dtype != torch.float32 or not bias.is_contiguous()):
+        raise ValueError("bias must be a contiguous fp32 tensor")
+    _check(_abi.load().lx_nvfp4_gemm(_ptr(xq.codes), _ptr(xq.sf), _ptr(xq.gscale), _ptr(wq.codes), _ptr(wq.sf),
+                                     _ptr(wq.gscale), _ptr(bias), M, N, K, _ptr(out), out.stride(0), _stream(stream)),
+           "lx_nvfp4_gemm")
+    return out
+
+
+def nvfp4_gemm_flops(M, N, K) -> float:
+    return 2.0 * M * N * K
 
 
 def lx_last_device_status(stream=None) -> int:

@@ -67,6 +67,9 @@ SIGNATURES = {
     "lx_ulysses_unpack_qkv": [_vp, _vp, _c_i64, _P(LxBhld), _P(LxBhld), _P(LxBhld), _vp],
     "lx_ulysses_pack_o": [_P(LxBhld), _c_i64, _vp, _vp, _vp],
     "lx_ulysses_unpack_o": [_vp, _vp, _c_i64, _c_i64, _c_i64, _P(LxBhld), _vp],
+    "lx_nvfp4_sizes": [_c_i64, _c_i64, _P(_c_sz), _P(_c_sz)],
+    "lx_nvfp4_quantize": [_vp, _c_i64, _c_i64, _c_i64, ctypes.c_int, _vp, _vp, _vp, _vp],
+    "lx_nvfp4_gemm": [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _c_i64, _c_i64, _c_i64, _vp, _c_i64, _vp],
     "lx_last_device_status": [_vp],
     "lx_debug_wait_timeout": [_u64, _vp],
     "lx_status_string": [ctypes.c_int],

@@ -12,6 +12,7 @@
 #include "planner.cuh"
 #include "quant.cuh"
 #include "ulysses.cuh"
+#include "nvfp4.cuh"
 #include "attn.cuh"
 
 namespace {
@@ -266,7 +267,7 @@ FwdWs fwd_layout(const lx_bhld* Q) {
 }  // namespace
 
 // ====================================================================== C ABI
-// Light-Ulysses launch helper (the entries are below, in the C block)
+// Light-Ulysses launch helper and the NVFP4 code map (the entries are below, in the C block)
 namespace {
 lx::BhldRW rw(const lx_bhld* t) {
   return lx::BhldRW{reinterpret_cast<__nv_bfloat16*>(t->data), t->sB, t->sH, t->sL};
@@ -286,6 +287,21 @@ lx_status launch_ulysses(lx::UlyssesArgs a, int64_t D, cudaStream_t s) {
     lx::ulysses_rows_kernel<64, MODE><<<grid, 256, 0, s>>>(a);
   return launch_status();
 }
+
+// 2-D byte map over NVFP4 codes [rows][K/2] (innermost first), 128-byte swizzle,
+// box of 128 bytes x box_rows rows; rows past the end read as zero.
+bool make_map_codes(CUtensorMap* m, const void* ptr, int64_t rows, int64_t K, int box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[2] = {(cuuint64_t)(K / 2), (cuuint64_t)rows};
+  const cuuint64_t strides[1] = {(cuuint64_t)(K / 2)};
+  const cuuint32_t box[2] = {128, (cuuint32_t)box_rows};
+  const cuuint32_t es[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(ptr), dims, strides, box, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 }  // namespace
 
 extern "C" {
@@ -773,4 +789,74 @@ lx_status lx_ulysses_unpack_o(const uint8_t* codes, const float* scales, int64_t
   return launch_ulysses<lx::kUnpackO>(a, out->D, stream);
 }
 
+// ---------------------------------------------------------------- NVFP4
+lx_status lx_nvfp4_sizes(int64_t R, int64_t K, size_t* code_bytes, size_t* sf_bytes) {
+  if (R < 1 || K < 64 || K % 64 != 0 || K > ((int64_t)1 << 30)) return LX_ERR_INVALID;
+  if (code_bytes) *code_bytes = (size_t)R * (size_t)(K / 2);
+  if (sf_bytes) *sf_bytes = (size_t)((R + 127) / 128) * 128 * (size_t)(K / 16);
+  return LX_OK;
+}
+
+lx_status lx_nvfp4_quantize(const void* x, int64_t R, int64_t K, int64_t ldx, int compute_gscale, float* gscale,
+                            uint8_t* codes, uint8_t* sf, cudaStream_t stream) {
+  if (!x || !gscale || !codes || !sf) return LX_ERR_INVALID;
+  if (R < 1 || K < 64 || K % 64 != 0 || K > ((int64_t)1 << 30) || ldx < K) return LX_ERR_INVALID;
+  const int64_t tiles = (R + 127) / 128, ysteps = (K / 64 + lx::kNvQSteps - 1) / lx::kNvQSteps;
+  if (tiles > 0x7FFFFFFF || ysteps > 65535) return LX_ERR_UNSUPPORTED;
+  if (!al16(x) || ldx % 8 != 0 || !al16(codes) || !al16(sf) || (reinterpret_cast<uintptr_t>(gscale) & 3u))
+    return LX_ERR_ALIGN;
+  const auto* xb = reinterpret_cast<const __nv_bfloat16*>(x);
+  if (compute_gscale) {
+    if (cudaMemsetAsync(gscale, 0, sizeof(float), stream) != cudaSuccess) return LX_ERR_CUDA;
+    int dev = 0, sms = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+      return LX_ERR_CUDA;
+    const int64_t ctas = R < 8LL * sms ? R : 8LL * sms;
+    lx::nvfp4_amax_kernel<<<(unsigned)ctas, 256, 0, stream>>>(xb, R, (int)K, ldx, reinterpret_cast<unsigned*>(gscale));
+    lx::nvfp4_gscale_kernel<<<1, 1, 0, stream>>>(gscale);
+  }
+  lx::nvfp4_quant_kernel<<<dim3((unsigned)tiles, (unsigned)ysteps), 128, 0, stream>>>(xb, R, (int)K, ldx, gscale,
+                                                                                       codes, sf);
+  return launch_status();
+}
+
+lx_status lx_nvfp4_gemm(const uint8_t* xc, const uint8_t* xsf, const float* gx, const uint8_t* wc,
+                        const uint8_t* wsf, const float* gw, const float* bias, int64_t M, int64_t N, int64_t K,
+                        void* y, int64_t ldy, cudaStream_t stream) {
+  if (!xc || !xsf || !gx || !wc || !wsf || !gw || !y) return LX_ERR_INVALID;
+  if (M < 1 || N < 128 || N % 128 != 0 || K < 256 || K % 256 != 0 || ldy < N) return LX_ERR_INVALID;
+  const int64_t mtiles = (M + lx::kNvBM - 1) / lx::kNvBM, ntiles = (N + lx::kNvBN - 1) / lx::kNvBN;
+  if (mtiles * ntiles > ((int64_t)1 << 40) || K > ((int64_t)1 << 30)) return LX_ERR_UNSUPPORTED;
+  if (!al16(xc) || !al16(xsf) || !al16(wc) || !al16(wsf) || !al16(y) || ldy % 8 != 0 ||
+      (reinterpret_cast<uintptr_t>(gx) & 3u) || (reinterpret_cast<uintptr_t>(gw) & 3u) ||
+      (reinterpret_cast<uintptr_t>(bias) & 3u))
+    return LX_ERR_ALIGN;
+  CUtensorMap ta, tw;
+  if (!make_map_codes(&ta, xc, M, K, lx::kNvBM) || !make_map_codes(&tw, wc, N, K, lx::kNvBN)) return LX_ERR_CUDA;
+  if (cudaFuncSetAttribute(lx::nvfp4_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)lx::kNvSmemBytes) !=
+      cudaSuccess)
+    return LX_ERR_CUDA;
+  lx::NvGemmArgs a{};
+  a.sfa = xsf;
+  a.sfb = wsf;
+  a.gx = gx;
+  a.gw = gw;
+  a.bias = bias;
+  a.y = reinterpret_cast<__nv_bfloat16*>(y);
+  a.ldy = ldy;
+  a.M = (int)M;
+  a.N = (int)N;
+  a.K = (int)K;
+  a.limit_ns = kWaitLimitNs;
+  int dev = 0, sms = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+      sms < 1)
+    return LX_ERR_CUDA;
+  const int64_t tiles = mtiles * ntiles;  // persistent: one CTA per SM walks the tiles
+  const unsigned grid = (unsigned)(tiles < sms ? tiles : sms);
+  lx::nvfp4_gemm_kernel<<<grid, lx::kNvThreads, lx::kNvSmemBytes, stream>>>(ta, tw, a);
+  return launch_status();
+}
+
 }  // extern "C"
+
