@@ -175,3 +175,25 @@ def test_smoothing_argument_errors_before_launch(lib):
     assert lib.lx_quantize_qk_smooth(ctypes.byref(k), ctypes.byref(k), 0x30008, *outs, s) == _abi.LX_ERR_ALIGN
     other = _view(L=999, H=2)
     assert lib.lx_quantize_qk_smooth(ctypes.byref(k), ctypes.byref(other), 0x30000, *outs, s) == _abi.LX_ERR_INVALID
+
+
+def test_nvfp4_sizes_and_argument_errors_before_launch(lib):
+    s = ctypes.c_void_p(0)
+    cb, sb = ctypes.c_size_t(), ctypes.c_size_t()
+    assert lib.lx_nvfp4_sizes(300, 320, ctypes.byref(cb), ctypes.byref(sb)) == 0
+    assert cb.value == 300 * 160
+    assert sb.value == oracle.sf_tiled(__import__("numpy").zeros((300, 20), "uint8")).size   # 3 tiles x 5 k-steps x 512
+    assert lib.lx_nvfp4_sizes(10, 96, ctypes.byref(cb), ctypes.byref(sb)) == _abi.LX_ERR_INVALID   # K % 64
+    assert lib.lx_nvfp4_sizes(0, 64, ctypes.byref(cb), ctypes.byref(sb)) == _abi.LX_ERR_INVALID
+    x, g, c, f = 0x10000, 0x20000, 0x30000, 0x40000
+    assert lib.lx_nvfp4_quantize(x, 10, 128, 100, 1, g, c, f, s) == _abi.LX_ERR_INVALID          # ldx < K
+    assert lib.lx_nvfp4_quantize(x, 10, 128, 132, 1, g, c, f, s) == _abi.LX_ERR_ALIGN            # ldx % 8
+    assert lib.lx_nvfp4_quantize(x + 8, 10, 128, 128, 1, g, c, f, s) == _abi.LX_ERR_ALIGN
+    assert lib.lx_nvfp4_quantize(None, 10, 128, 128, 1, g, c, f, s) == _abi.LX_ERR_INVALID
+    args = (c, f, g, c, f, g, None)
+    assert lib.lx_nvfp4_gemm(*args, 100, 256, 320, x, 256, s) == _abi.LX_ERR_INVALID             # K % 256
+    assert lib.lx_nvfp4_gemm(*args, 100, 192, 256, x, 192, s) == _abi.LX_ERR_INVALID             # N % 128
+    assert lib.lx_nvfp4_gemm(*args, 100, 256, 256, x, 200, s) == _abi.LX_ERR_INVALID             # ldy < N
+    assert lib.lx_nvfp4_gemm(*args, 100, 256, 256, x, 260, s) == _abi.LX_ERR_ALIGN               # ldy % 8
+    assert lib.lx_nvfp4_gemm(c, f, g + 2, c, f, g, None, 100, 256, 256, x, 256, s) == _abi.LX_ERR_ALIGN
+    assert lib.lx_nvfp4_gemm(c, None, g, c, f, g, None, 100, 256, 256, x, 256, s) == _abi.LX_ERR_INVALID
