@@ -309,7 +309,7 @@ lx_status lx_nvfp4_sizes(int64_t R, int64_t K, size_t* code_bytes, size_t* sf_by
 /* Quantise bf16 x [R, K] (row stride ldx elements, ldx % 8 == 0, K % 64 == 0,
  * 16-byte aligned) to NVFP4.  compute_gscale != 0: *gscale (device fp32) is
  * computed from x and written (an amax pass, then the quantiser); 0: *gscale
- * is read as given.  codes / sf: buffers of lx_nvfp4_sizes bytes, 16-byte
+ * is read as given and must be a positive finite fp32.  codes / sf: buffers of lx_nvfp4_sizes bytes, 16-byte
  * aligned, owned by the caller.  Finite inputs only. */
 lx_status lx_nvfp4_quantize(const void* x, int64_t R, int64_t K, int64_t ldx, int compute_gscale, float* gscale,
                             uint8_t* codes, uint8_t* sf, cudaStream_t stream);
@@ -319,8 +319,9 @@ lx_status lx_nvfp4_quantize(const void* x, int64_t R, int64_t K, int64_t ldx, in
  * block scale): X = (xc, xsf, gx) [M, K], W = (wc, wsf, gw) [N, K] as written by
  * lx_nvfp4_quantize; bias fp32 [N] or NULL; y bf16 [M, N] with row stride ldy
  * (ldy % 8 == 0, 16-byte aligned).  N % 128 == 0, K % 256 == 0; M is any
- * count >= 1 up to 65535*128.  A wait that runs out sets the device status
- * to LX_ERR_TIMEOUT (see lx_last_device_status). */
+ * count >= 1; M and N below 2^31 - 256, K up to 2^30 (else LX_ERR_UNSUPPORTED).
+ * One persistent CTA per SM walks the 128 x 256 output tiles.  A wait that
+ * runs out sets the device status to LX_ERR_TIMEOUT (see lx_last_device_status). */
 lx_status lx_nvfp4_gemm(const uint8_t* xc, const uint8_t* xsf, const float* gx, const uint8_t* wc,
                         const uint8_t* wsf, const float* gw, const float* bias, int64_t M, int64_t N, int64_t K,
                         void* y, int64_t ldy, cudaStream_t stream);

@@ -197,3 +197,4 @@ def test_nvfp4_sizes_and_argument_errors_before_launch(lib):
     assert lib.lx_nvfp4_gemm(*args, 100, 256, 256, x, 260, s) == _abi.LX_ERR_ALIGN               # ldy % 8
     assert lib.lx_nvfp4_gemm(c, f, g + 2, c, f, g, None, 100, 256, 256, x, 256, s) == _abi.LX_ERR_ALIGN
     assert lib.lx_nvfp4_gemm(c, None, g, c, f, g, None, 100, 256, 256, x, 256, s) == _abi.LX_ERR_INVALID
+    assert lib.lx_nvfp4_gemm(*args, 1 << 31, 256, 256, x, 256, s) == _abi.LX_ERR_UNSUPPORTED       # 32-bit rows

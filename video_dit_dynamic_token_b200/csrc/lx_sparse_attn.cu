@@ -826,7 +826,9 @@ lx_status lx_nvfp4_gemm(const uint8_t* xc, const uint8_t* xsf, const float* gx, 
   if (!xc || !xsf || !gx || !wc || !wsf || !gw || !y) return LX_ERR_INVALID;
   if (M < 1 || N < 128 || N % 128 != 0 || K < 256 || K % 256 != 0 || ldy < N) return LX_ERR_INVALID;
   const int64_t mtiles = (M + lx::kNvBM - 1) / lx::kNvBM, ntiles = (N + lx::kNvBN - 1) / lx::kNvBN;
-  if (mtiles * ntiles > ((int64_t)1 << 40) || K > ((int64_t)1 << 30)) return LX_ERR_UNSUPPORTED;
+  // row and column coordinates of the TMA loads and the kernel's sizes are 32-bit
+  if (M > ((int64_t)1 << 31) - 256 || N > ((int64_t)1 << 31) - 256 || K > ((int64_t)1 << 30))
+    return LX_ERR_UNSUPPORTED;
   if (!al16(xc) || !al16(xsf) || !al16(wc) || !al16(wsf) || !al16(y) || ldy % 8 != 0 ||
       (reinterpret_cast<uintptr_t>(gx) & 3u) || (reinterpret_cast<uintptr_t>(gw) & 3u) ||
       (reinterpret_cast<uintptr_t>(bias) & 3u))
