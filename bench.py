@@ -447,7 +447,7 @@ def run_nvfp4_gemm(args):
 
     dev = torch.device("cuda", 0)
     torch.cuda.set_device(dev)
-    M, N, K = (args.gemm_m or 75600), 15360, 5120
+    M, N, K = (args.gemm_m or 75600), (args.gemm_n or 15360), (args.gemm_k or 5120)
     g = torch.Generator(device=dev).manual_seed(0)
     X = torch.randn((M, K), generator=g, device=dev).to(torch.bfloat16)
     W = (torch.randn((N, K), generator=g, device=dev) * 0.02).to(torch.bfloat16)
@@ -496,8 +496,9 @@ def run_nvfp4_gemm(args):
            "warmup": max(3, args.warmup), "ms_per_step": round(ms, 4), "higher_is_better": True, "scaling": "weak",
            "vs_baseline": None, "dtype": "nvfp4 (e2m1 x e2m1, e4m3/16 scales, f32 accumulate, bf16 out)",
            "data": "synthetic: X ~ N(0,1), W ~ N(0, 0.02^2), bias ~ N(0, 0.01)",
-           "config": {"workload": GEMM_WORKLOAD if M == 75600 else f"NVFP4 QKV projection, M={M}, K={K}, N={N}",
-                      "M": M, "N": N, "K": K, "l2": "inputs larger than L2 (X 774 MB)"},
+           "config": {"workload": GEMM_WORKLOAD if (M, N, K) == (75600, 15360, 5120)
+                      else f"NVFP4 linear layer, M={M}, K={K}, N={N}",
+                      "M": M, "N": N, "K": K, "l2": f"inputs larger than L2 (X {M * K * 2 / 1e6:.0f} MB)"},
            "breakdown_ms": {"quantise_x": round(q_ms, 4), "gemm": round(g_ms, 4)},
            "roofline": {"bound": "tensor", "achieved": round(flops / (g_ms * 1e-3) / 1e12, 1),
                         "peak": round(fp4_peak, 1), "unit": "TFLOP/s",
@@ -513,8 +514,8 @@ def run_nvfp4_gemm(args):
            "note": "sub-benchmark of the NVFP4 projection kernel; the headline line (no flags) carries e2e"}
     if not args.no_cpu_baseline:
         out["cpu_baseline"] = nvfp4_cpu_sample(M, N, K)
-    if M != 75600:
-        out["note"] = "smaller M: a profiling case, not the benchmark"
+    if (M, N, K) != (75600, 15360, 5120):
+        out["note"] = "another shape: a characterisation or profiling case, not the benchmark"
     return out
 
 # ------------------------------------------------------------------ CPU oracle timing
@@ -602,7 +603,9 @@ def main():
                     help="int8fp8: the Q/K pass also applies per-head RMSNorm and 3D RoPE (lx_qk_prologue)")
     ap.add_argument("--gemm", action="store_true",
                     help="time one NVFP4 linear layer (the 720p fused QKV projection) instead")
-    ap.add_argument("--gemm-m", type=int, default=0, help="--gemm with fewer token rows: a profiling case only")
+    ap.add_argument("--gemm-m", type=int, default=0, help="--gemm with another token count (profiling)")
+    ap.add_argument("--gemm-n", type=int, default=0, help="--gemm with another output width (characterisation)")
+    ap.add_argument("--gemm-k", type=int, default=0, help="--gemm with another input width (characterisation)")
     args = ap.parse_args()
     if args.gemm:
         print(json.dumps(run_nvfp4_gemm(args)))
