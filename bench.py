@@ -330,6 +330,42 @@ def run_ours(args, rank, world, local_rank):
 
 
 # ------------------------------------------------------------------ Light-Ulysses share
+def attn_roofline(flops, ms, peaks, mode, d):
+    """The attention kernel against the dense 8-bit (2x sustained bf16) or bf16 peak."""
+    peak = (2.0 if mode == "int8fp8" else 1.0) * peaks["bf16_sustained"]
+    achieved = flops / (ms * 1e-3) / 1e12
+    return {"bound": "tensor", "kernel": f"sparse_attn_kernel<{d},{mode}>", "achieved": round(achieved, 1),
+            "peak": round(peak, 1), "unit": "TFLOP/s", "frac": round(achieved / peak, 3), "traffic": None,
+            "peak_note": f"{'2 x ' if mode == 'int8fp8' else ''}{peaks['source']} sustained bf16 "
+                         f"({peaks['bf16_sustained']})"}
+
+
+def ulysses_cpu_sample(N, B, H, d, L, flops, sample_tokens=256, attn=None):
+    """The oracle on a bounded sample of one rank's share: the exchange steps
+    (pack/unpack of the Q/K/V payload and of the output) on `sample_tokens` of
+    the shard's tokens, scaled to the shard, plus the attention at the oracle's
+    sampled rate (cpu_oracle_sample, or `attn` when given)."""
+    import numpy as np
+
+    import oracle
+    Hr, Lr = H // N, L // N
+    rng = np.random.default_rng(0)
+    ts = min(sample_tokens, Lr)
+    q, k, v = (rng.standard_normal((B, ts, H, d)).astype(np.float32) for _ in range(3))
+    o = rng.standard_normal((B, Hr, N * ts, d)).astype(np.float32)
+    t0 = time.perf_counter()
+    c, sc = oracle.pack_qkv_ref(q, k, v, N)
+    oracle.unpack_qkv_ref(c, sc)            # the send buffer stands in for the received one
+    oc, osc = oracle.pack_o_ref(o, N)
+    oracle.unpack_o_ref(oc, osc)
+    t_x = (time.perf_counter() - t0) * (Lr / ts)
+    attn = attn or cpu_oracle_sample()
+    t_attn = flops / (attn["value"] * 1e12)
+    return {"value": flops / (t_attn + t_x) / 1e12, "unit": "TFLOP/s", "cores": attn["cores"], "kind": "oracle",
+            "sample": f"exchange steps on {ts} of the shard's {Lr} tokens ({t_x * ts / Lr:.2f} s, scaled x{Lr / ts:.0f}); "
+                      f"attention at the oracle's sampled rate ({attn['sample']})"}
+
+
 def run_ulysses_share(args):
     """One rank's share of an N-GPU Light-Ulysses step at the workload's grid,
     timed on one GPU: pack this rank's token shard (all heads) into the FP8
@@ -386,11 +422,14 @@ def run_ulysses_share(args):
     torch.cuda.synchronize()
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(args.steps)]
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler(0)
+    sampler.start()
     t0.record()
     for i in range(args.steps):
         step(evs[i])
     t1.record()
     torch.cuda.synchronize()
+    clocks = sampler.stop()
     if lx.lx_last_device_status() != 0:
         raise RuntimeError("device status error")
     ms = t0.elapsed_time(t1) / args.steps
@@ -409,6 +448,9 @@ def run_ulysses_share(args):
             "data": "synthetic N(0,1) shards", "config": {"workload": f"{args.workload} B={B} H={H} d={d} L={L} N={N}",
                                                           "shard_tokens": Lr, "heads_after_exchange": Hr},
             "breakdown_ms": {n: round(v, 4) for n, v in per.items()}, "phases": phases,
+            "roofline": attn_roofline(flops, per["attn"], peaks, args.mode, d),
+            "gpu_launches": (10 if args.mode == "int8fp8" else 8) * args.steps, "clocks": clocks, "e2e": None,
+            "cpu_baseline": (None if args.no_cpu_baseline else ulysses_cpu_sample(N, B, H, d, L, flops)),
             "note": "the all-to-all is not timed (one GPU); the send buffer stands in for the received one"}
 
 
