@@ -199,3 +199,35 @@ def test_quant_k_smooth_rule():
             want = int(np.clip(np.rint(np.float32(x[t, c] * inv)), -127, 127))
             assert codes[0, 0, t, c] == want
     assert scales[0, 0, 0] == np.float32(a / np.float32(127.0))
+
+
+def test_prologue_output_scalar_brute_force():
+    """Y of a few rows re-derived with scalar loops: the RMS over the head's
+    channels, the weight, then each channel pair turned by position * theta^(-2i/m)
+    of its part (math.cos / math.sin), then the bf16 rounding of torch's cast."""
+    d, grid, eps, theta = 64, (3, 4, 5), 1e-6, 10000.0
+    x = _rand((1, 2, 60, d), 11, scale=2.0)
+    w = 1.0 + 0.2 * _rand((2, d), 12)
+    Y = oracle.prologue_ref(x, w, eps, grid, theta)["Y"]
+    parts = (d - 4 * (d // 6), 2 * (d // 6), 2 * (d // 6))
+    T, Hh, W = grid
+    for h, t in [(0, 0), (1, 7), (0, 33), (1, 59)]:
+        row = x[0, h, t].astype(np.float64)
+        rms = math.sqrt(sum(v * v for v in row) / d + eps)
+        y = [row[c] / rms * w[h, c] for c in range(d)]
+        pos = (t // (Hh * W), (t // W) % Hh, t % W)
+        out, c0 = list(y), 0
+        for axis, m in enumerate(parts):
+            for i in range(m // 2):
+                ang = pos[axis] * theta ** (-2.0 * i / m)
+                a, b = y[c0 + 2 * i], y[c0 + 2 * i + 1]
+                out[c0 + 2 * i] = a * math.cos(ang) - b * math.sin(ang)
+                out[c0 + 2 * i + 1] = a * math.sin(ang) + b * math.cos(ang)
+            c0 += m
+        want = torch.tensor(out, dtype=torch.float32).to(torch.bfloat16).double().numpy()
+        got = Y[0, h, t]
+        # torch rounds the fp32 value, the oracle the fp64 one: equal except where
+        # the fp32 rounding lands on a bf16 tie, which one ulp covers
+        ulp = np.ldexp(1.0, np.floor(np.log2(np.maximum(np.abs(want), 1e-30))).astype(int) - 7)
+        assert np.all(np.abs(got - want) <= ulp)
+        assert np.mean(got == want) > 0.95

@@ -82,3 +82,13 @@ def test_exchange_layout_against_brute_force(N):
                 for t in range(Lr):
                     c, s = oracle.fp8_rows_ref(o[src][:, h, r * Lr + t, :])
                     assert np.array_equal(got[:, t, src * (H // N) + h, :], oracle.fp8_rows_dequant_ref(c, s))
+
+
+def test_dequant_is_bf16_of_the_fp32_product():
+    """The receiver's value is bf16(fl32(decode(code) * scale)), with torch's fp32
+    product and its round-to-nearest-even bf16 cast as the reference."""
+    x = torch.from_numpy(_rand((6, 64), 3, scale=7.0)).to(torch.bfloat16)
+    codes, scales = oracle.fp8_rows_ref(x)
+    dec = torch.from_numpy(codes).view(torch.float8_e4m3fn).float()
+    want = (dec * torch.from_numpy(scales)[:, None]).to(torch.bfloat16).double().numpy()
+    assert np.array_equal(oracle.fp8_rows_dequant_ref(codes, scales), want)
