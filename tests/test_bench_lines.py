@@ -23,3 +23,34 @@ def test_ulysses_cpu_sample_combines_exchange_and_attention():
     # the exchange adds time, so the rate is below the attention-only rate
     assert 0 < r["value"] < 1e-3
     assert "64 of the shard's 256 tokens" in r["sample"]
+
+
+class _FakeProc:
+    def terminate(self):
+        pass
+
+    def wait(self, timeout=None):
+        return 0
+
+
+def _sampler_with(lines):
+    s = bench.ClockSampler(0)
+    s.proc = _FakeProc()
+    s.lines = list(lines)
+    return s.stop()
+
+
+def test_clock_sampler_median_and_reasons():
+    base = "0, {mhz}, 1965, 700.5, 0x0, {hw}, Not Active, Not Active, {pc}"
+    lines = [base.format(mhz=m, hw="Not Active", pc="Not Active") for m in (1965, 1950, 1965)]
+    r = _sampler_with(lines)
+    assert r["sm_mhz"] == 1965.0 and r["sm_max_mhz"] == 1965.0 and r["reasons"] == [] and r["samples"] == 3
+    lines.append(base.format(mhz=1500, hw="Active", pc="Active"))
+    r = _sampler_with(lines)
+    assert r["reasons"] == ["hw_slowdown", "sw_power_cap"]
+    assert r["samples"] == 4 and r["sm_mhz"] == 1965.0
+
+
+def test_clock_sampler_ignores_malformed_lines():
+    r = _sampler_with(["garbage", "0, [N/A], 1965, 1, 0, a, b, c, d", ""])
+    assert r["sm_mhz"] is None and r["samples"] == 0
