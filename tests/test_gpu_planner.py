@@ -97,7 +97,8 @@ def test_plan_parity_full_size(name):
     assert lx.lx_last_device_status() == 0
     Qc, Kc = Q.cpu(), K.cpu()
     del Q, K
-    check_plan(plan.idx, plan.mask, Qc, Kc, w.keep)
+    # a flipped pair costs two bits; near-ties at the k-th place are rare
+    check_plan(plan.idx, plan.mask, Qc, Kc, w.keep, max_exempt_frac=2e-3)
 
 
 @pytest.mark.parametrize("keep", [0.05, 0.5, 1.0])
@@ -107,7 +108,7 @@ def test_plan_parity_720p_keep_sweep(keep, smooth):
     Q, K, _ = synth.make_qkv(1, 4, w.d, w.grid, seed=1, smooth=smooth, device=DEV)
     plan = lx.lx_sparse_attn_plan(Q, K, keep)
     assert lx.lx_last_device_status() == 0
-    check_plan(plan.idx, plan.mask, Q.cpu(), K.cpu(), keep)
+    check_plan(plan.idx, plan.mask, Q.cpu(), K.cpu(), keep, max_exempt_frac=2e-3)
 
 
 @pytest.mark.parametrize("keep", [0.1, 0.5])

@@ -418,3 +418,76 @@ def test_int8fp8_close_to_exact_on_smooth_field():
     O8 = oracle.attn_ref_int8fp8(Q, K, V, p["idx"])
     O = oracle.attn_ref_exact(Q, K, V, p["idx"])
     assert oracle.rel_l1_err(O8, O) < 0.08
+
+
+# ---------------------------------------------------------------- threshold and error measures
+def _kth_by_repeated_removal(row, k):
+    """The k-th largest value of a list, found by removing the maximum k-1 times."""
+    vals = [float(v) for v in row]
+    for _ in range(k - 1):
+        vals.remove(max(vals))
+    return max(vals)
+
+
+@pytest.mark.parametrize("k", [1, 2, 3, 5, 8])
+def test_kth_threshold_against_repeated_removal(k):
+    # Rows built with ties exactly at the k-th place, negative rows, and one
+    # row of equal scores; the threshold is the k-th largest value counted with
+    # multiplicity (the score the k-th kept block has).
+    rows = np.array([
+        [0.5, 3.0, 3.0, 1.0, -2.0, 3.0, 0.0, 7.0],
+        [-1.0, -4.0, -0.5, -0.5, -9.0, -3.0, -0.5, -2.0],
+        [2.0, 2.0, 2.0, 2.0, 2.0, 2.0, 2.0, 2.0],
+        [1e-9, -1e-9, 0.0, 5.0, 5.0, 4.0, 4.0, 4.0],
+    ])
+    got = oracle.kth_threshold(rows, k)
+    want = np.array([_kth_by_repeated_removal(r, k) for r in rows])
+    assert np.array_equal(got, want)
+    # the selection keeps exactly the blocks with a score above tau, plus the
+    # lowest-index ones among those equal to tau
+    sel = oracle.select_topk(rows, k)
+    for r in range(rows.shape[0]):
+        tau = want[r]
+        assert np.all(rows[r][sel[r]] >= tau)
+        assert np.sum(rows[r] > tau) <= k
+
+
+def test_kth_threshold_ends_of_the_range():
+    rng = np.random.default_rng(3)
+    s = rng.standard_normal((2, 3, 5, 13))
+    # k = 1 is the row maximum, k = nB the row minimum
+    assert np.array_equal(oracle.kth_threshold(s, 1), s.max(axis=-1))
+    assert np.array_equal(oracle.kth_threshold(s, 13), s.min(axis=-1))
+    # a hand-computed row: sorted descending 9, 7, 7, 4, 1 -> k = 2, 3 give 7, k = 4 gives 4
+    row = np.array([[4.0, 7.0, 1.0, 9.0, 7.0]])
+    assert [float(oracle.kth_threshold(row, k)[0]) for k in (1, 2, 3, 4, 5)] == [9.0, 7.0, 7.0, 4.0, 1.0]
+
+
+def test_error_measures_hand_computed():
+    # Values worked by hand.  O - R = [0.5, -1, 0, 0.25, -0.125, 0.5]; |R| sums to
+    # 1 + 2 + 0 + 4 + 0.5 + 0.5 = 8, so rel-L1 = (0.5 + 1 + 0 + 0.25 + 0.125 + 0.5) / 8
+    # = 2.375 / 8 = 0.296875.  A reference entry of 0 contributes its error to the
+    # numerator and nothing to the denominator; no element-wise ratio is taken.
+    R = np.array([[1.0, -2.0, 0.0], [4.0, 0.5, -0.5]])
+    O = np.array([[1.5, -3.0, 0.0], [4.25, 0.375, 0.0]])
+    assert oracle.max_abs_err(O, R) == 1.0
+    assert oracle.rel_l1_err(O, R) == 0.296875
+    # symmetric in the sign of the error, exact zero for equal arrays
+    assert oracle.max_abs_err(R, O) == 1.0
+    assert oracle.max_abs_err(R, R) == 0.0 and oracle.rel_l1_err(R, R) == 0.0
+    # the measure is over all elements, not per row: a row-wise mean of ratios
+    # would give (1.5/3 + 0.875/5) / 2 = 0.3375 here
+    assert oracle.rel_l1_err(O, R) != 0.3375
+    # a large error at the single zero reference entry stays finite
+    O2 = R.copy()
+    O2[0, 2] = 3.0
+    assert oracle.rel_l1_err(O2, R) == 3.0 / 8.0
+    assert oracle.max_abs_err(O2, R) == 3.0
+
+
+def test_error_measures_accept_torch_and_bf16():
+    R = torch.tensor([[0.5, -1.5], [2.0, 0.0]], dtype=torch.float64)
+    O = torch.tensor([[0.5, -1.0], [2.0, 0.25]], dtype=torch.bfloat16)
+    # bf16 holds these values exactly: |O - R| = [0, 0.5, 0, 0.25], sum |R| = 4
+    assert oracle.max_abs_err(O, R) == 0.5
+    assert oracle.rel_l1_err(O, R) == 0.75 / 4.0
