@@ -36,11 +36,33 @@ def metric_for(workload, H, d, keep):
     return f"block-sparse attn ms & effective TFLOPS ({workload} grid, {H}\u00d7{d}, keep {keep:g})"
 
 
-# DRAM bytes (read + write) of one full-size attention launch of the current
-# kernel build: the ncu capture in profiles/attn_int8fp8_720p_8heads_ncu.md
-# (8 of the 40 heads; traffic grows with the head count, so x5).  Set to None
-# whenever the attention kernel changes until it is captured again.
-ATTN_DRAM_BYTES_PER_LAUNCH = 5 * (236.903424e6 + 126.946048e6)
+# DRAM bytes (read + write) of one full-size attention launch, from an ncu
+# capture, keyed by the SHA-256 of the kernel source it was taken on: when
+# attn.cuh changes the key no longer matches and the line reports null.
+ATTN_SRC = os.path.join(ROOT, "video_dit_dynamic_token_b200", "csrc", "attn.cuh")
+ATTN_DRAM_BYTES = {   # {sha256 of attn.cuh: (bytes per full 720p launch, how it was taken)}
+    "05b326c7b53ef8e933eb51083a6ff51c0abb28fbb8a2ea0d641653828126b804":
+        (5 * (236.935168e6 + 126.793984e6),
+         "ncu dram__bytes_read.sum + dram__bytes_write.sum of the 8-head 720p launch x 5 (traffic grows with the "
+         "heads)"),
+}
+
+# Dense MACs per clock per SM of one tcgen05 kind::i8 / kind::f8f6f4 M=128 MMA
+# stream, measured with back-to-back MMAs on this chip (8170 of 8192).
+TC_8BIT_MAC_PER_CLK_SM = 8192
+PEAKS_8BIT = os.path.join(ROOT, "MEASURED_PEAKS_8BIT.json")
+
+
+def attn_traffic():
+    import hashlib
+    try:
+        h = hashlib.sha256(open(ATTN_SRC, "rb").read()).hexdigest()
+    except OSError:
+        return None, "kernel source not found"
+    if h in ATTN_DRAM_BYTES:
+        b, how = ATTN_DRAM_BYTES[h]
+        return int(b), how
+    return None, "no ncu capture of this kernel source yet"
 
 
 def reduce_max(x: float, device) -> float:
@@ -63,9 +85,98 @@ def _peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
         d = json.load(open(p))
-        return {"hbm_gbs": d["hbm_gbs"], "bf16": d["bf16_tflops"], "bf16_sustained": d["bf16_tflops_sustained"],
-                "source": "measured"}
-    return {"hbm_gbs": 6650.0, "bf16": 1590.0, "bf16_sustained": 1400.0, "source": "fallback"}
+        out = {"hbm_gbs": d["hbm_gbs"], "bf16": d["bf16_tflops"], "bf16_sustained": d["bf16_tflops_sustained"],
+               "source": "measured"}
+    else:
+        out = {"hbm_gbs": 6650.0, "bf16": 1590.0, "bf16_sustained": 1400.0, "source": "fallback"}
+    # dense 8-bit peaks (cuBLAS int8 and fp8 GEMMs, `bench.py --peaks`); until
+    # measured, 2 x the bf16 burst figure (the nominal ratio)
+    if os.path.exists(PEAKS_8BIT):
+        e = json.load(open(PEAKS_8BIT))
+        out["int8"], out["fp8"] = e["int8_tops"], e["fp8_tflops"]
+        out["int8_sustained"], out["fp8_sustained"] = e["int8_tops_sustained"], e["fp8_tflops_sustained"]
+        out["source_8bit"] = "measured (MEASURED_PEAKS_8BIT.json)"
+    else:
+        out["int8"] = out["fp8"] = 2.0 * out["bf16"]
+        out["int8_sustained"] = out["fp8_sustained"] = 2.0 * out["bf16_sustained"]
+        out["source_8bit"] = f"2 x {out['source']} bf16 (nominal ratio)"
+    return out
+
+
+def attn_roofline(flops, ms, peaks, mode, d, sm_mhz=None, sms=148):
+    """The attention kernel's effective TFLOP/s against the dense peak of its
+    dtype: the 8-bit GEMM burst peak (the larger of int8 and fp8; the kernel
+    is timed alone for well under a second) or bf16, plus the sustained
+    figure and the tcgen05 MMA rate at the sampled clock as second fields."""
+    achieved = flops / (ms * 1e-3) / 1e12
+    if mode == "int8fp8":
+        peak = max(peaks["int8"], peaks["fp8"])
+        sustained = max(peaks["int8_sustained"], peaks["fp8_sustained"])
+        note = f"dense 8-bit burst, {peaks['source_8bit']}: int8 {peaks['int8']}, fp8 {peaks['fp8']}"
+        mac = TC_8BIT_MAC_PER_CLK_SM
+    else:
+        peak, sustained = peaks["bf16"], peaks["bf16_sustained"]
+        note = f"{peaks['source']} bf16 burst"
+        mac = TC_8BIT_MAC_PER_CLK_SM // 2
+    out = {"bound": "tensor", "kernel": f"sparse_attn_kernel<{d},{mode}>", "achieved": round(achieved, 1),
+           "peak": round(peak, 1), "unit": "TFLOP/s", "frac": round(achieved / peak, 3), "peak_note": note,
+           "frac_of_sustained": round(achieved / sustained, 3), "sustained_peak": round(sustained, 1)}
+    if sm_mhz:
+        tc = 2.0 * mac * sms * sm_mhz * 1e6 / 1e12
+        out["tcgen05_peak_at_clock"] = round(tc, 1)
+        out["frac_of_tcgen05_at_clock"] = round(achieved / tc, 3)
+    return out
+
+
+def measure_8bit_peaks(seconds=4.0, n=8192):
+    """Dense int8 (torch._int_mm) and fp8 e4m3 (torch._scaled_mm) GEMM peaks on
+    this GPU: the best of 10 single launches (burst) and back-to-back launches
+    for `seconds` (sustained), 2*n^3 operations each; nvidia-smi clocks sampled
+    during the sustained loops."""
+    import torch
+    dev = torch.device("cuda", 0)
+    g = torch.Generator(device=dev).manual_seed(0)
+    a8 = torch.randint(-64, 64, (n, n), generator=g, device=dev, dtype=torch.int8)
+    b8 = torch.randint(-64, 64, (n, n), generator=g, device=dev, dtype=torch.int8).t()   # column-major B
+    af = torch.randn(n, n, generator=g, device=dev).to(torch.float8_e4m3fn)
+    bf = torch.randn(n, n, generator=g, device=dev).to(torch.float8_e4m3fn).t()
+    one = torch.ones((), device=dev)
+    ops = {"int8": lambda: torch._int_mm(a8, b8),
+           "fp8": lambda: torch._scaled_mm(af, bf, scale_a=one, scale_b=one, out_dtype=torch.bfloat16)}
+    flop = 2.0 * n ** 3
+    res = {}
+    for name, f in ops.items():
+        for _ in range(3):
+            f()
+        torch.cuda.synchronize()
+        best = float("inf")
+        for _ in range(10):
+            s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            s.record()
+            f()
+            e.record()
+            torch.cuda.synchronize()
+            best = min(best, s.elapsed_time(e))
+        sampler = ClockSampler(0)
+        sampler.start()
+        time.sleep(0.2)
+        s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        reps = max(1, int(seconds / (best * 1e-3)))
+        s.record()
+        for _ in range(reps):
+            f()
+        e.record()
+        torch.cuda.synchronize()
+        clk = sampler.stop()
+        res[name] = {"burst": flop / (best * 1e-3) / 1e12,
+                     "sustained": flop * reps / (s.elapsed_time(e) * 1e-3) / 1e12, "clocks": clk}
+    return {"int8_tops": round(res["int8"]["burst"], 1), "int8_tops_sustained": round(res["int8"]["sustained"], 1),
+            "fp8_tflops": round(res["fp8"]["burst"], 1), "fp8_tflops_sustained": round(res["fp8"]["sustained"], 1),
+            "clocks_int8_sustained": res["int8"]["clocks"], "clocks_fp8_sustained": res["fp8"]["clocks"],
+            "gpu_name": torch.cuda.get_device_name(dev), "torch": torch.__version__,
+            "how": f"torch._int_mm (int8 x int8 -> int32) and torch._scaled_mm (e4m3 x e4m3 -> bf16, unit scales), "
+                   f"{n}^3, 2*n^3 operations: best of 10 single launches (burst) and back to back for "
+                   f"{seconds:g} s (sustained)"}
 
 
 class ClockSampler:
@@ -245,6 +356,25 @@ def run_ours(args, rank, world, local_rank):
     ms_step = total_ms / args.steps
     value = job_tflops(world, flops, ms_step)
 
+    # ---- the planner alone (a1 + a2: block means, scores, top-k) as a user
+    # calls it, for its HBM roofline: Q and K read once, the plan written once
+    pl_ms = None
+    if args.planner_steps > 0:
+        for _ in range(2):
+            lx.lx_sparse_attn_plan(Q, K, keep, plan=plan, ws=plan_ws)
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(args.planner_steps):
+            lx.lx_sparse_attn_plan(Q, K, keep, plan=plan, ws=plan_ws)
+        b.record(stream)
+        torch.cuda.synchronize()
+        pl_ms = reduce_max(a.elapsed_time(b) / args.planner_steps, dev)
+        if lx.lx_last_device_status() != 0:
+            raise RuntimeError("device status error in the planner leg")
+
     # ---- end to end through the public API with host buffers
     e2e = None
     if args.e2e_steps > 0:
@@ -278,8 +408,6 @@ def run_ours(args, rank, world, local_rank):
     peaks = _peaks()
     attn_ms = per["attn"]
     achieved = flops / (attn_ms * 1e-3) / 1e12
-    # dense 8-bit peak = 2 x bf16 (the nominal ratio); bf16 mode against bf16 itself
-    peak = (2.0 if mode == "int8fp8" else 1.0) * peaks["bf16_sustained"]
     # algorithmic HBM bytes of the phases before attention (each tensor once per
     # pass that must touch it; the block means and scores are small or L2-sized)
     N = B * H * L * d
@@ -297,9 +425,22 @@ def run_ours(args, rank, world, local_rank):
     phases = {n: {"ms": round(per[n], 4), "algorithmic_mb": round(b / 1e6, 1),
                   "gbs": round(b / (per[n] * 1e-3) / 1e9, 1),
                   "hbm_frac": round(b / (per[n] * 1e-3) / 1e9 / peaks["hbm_gbs"], 3)} for n, b in phase_bytes.items()}
+    if pl_ms is not None:
+        # the planner's algorithmic bytes: Q and K read once, idx and mask written once
+        pb = 2 * N * 2 + plan_out_b
+        phases["planner"] = {"ms": round(pl_ms, 4), "algorithmic_mb": round(pb / 1e6, 1),
+                             "gbs": round(pb / (pl_ms * 1e-3) / 1e9, 1),
+                             "hbm_frac": round(pb / (pl_ms * 1e-3) / 1e9 / peaks["hbm_gbs"], 3),
+                             "call": "lx_sparse_attn_plan (block means, score GEMM, top-k), timed alone",
+                             "of_8tbs_spec": round(pb / (pl_ms * 1e-3) / 1e9 / 8000.0, 3)}
     # Q/K/V (codes or bf16) read once, O written once (bf16), kept ids
     esz = 1 if mode == "int8fp8" else 2
     attn_bytes = 3 * B * H * L * d * esz + B * H * L * d * 2 + B * H * nB * k * 4
+    roof = attn_roofline(flops, attn_ms, peaks, mode, d, (clocks or {}).get("sm_mhz"))
+    traffic, traffic_note = attn_traffic()
+    if args.heads or mode != MODE or args.workload != WORKLOAD or args.keep:
+        traffic, traffic_note = None, "captured for the 720p headline launch only"
+    roof.update({"traffic": traffic, "traffic_note": traffic_note, "algorithmic_bytes": int(attn_bytes)})
     out = {
         "metric": metric_for(args.workload, H, d, keep), "value": round(value, 2), "unit": "TFLOP/s",
         "n_gpus": world, "steps": args.steps,
@@ -312,17 +453,10 @@ def run_ours(args, rank, world, local_rank):
         "breakdown_ms": {n: round(v, 4) for n, v in per.items()},
         "attn_ms": round(attn_ms, 4), "attn_effective_tflops": round(achieved, 1),
         "phases": phases,
-        "roofline": {"bound": "tensor", "kernel": f"sparse_attn_kernel<{d},{mode}>", "achieved": round(achieved, 1),
-                     "peak": round(peak, 1), "unit": "TFLOP/s", "frac": round(achieved / peak, 3),
-                     "peak_note": (f"2 x {peaks['source']} sustained bf16 ({peaks['bf16_sustained']}) = dense "
-                                   "int8/fp8 by the nominal 2:1 ratio" if mode == "int8fp8" else
-                                   f"{peaks['source']} sustained bf16 ({peaks['bf16_sustained']})"),
-                     "traffic": (None if ATTN_DRAM_BYTES_PER_LAUNCH is None or args.heads or mode != MODE
-                                 or args.workload != WORKLOAD or args.keep
-                                 else int(ATTN_DRAM_BYTES_PER_LAUNCH)),
-                     "traffic_note": "ncu dram__bytes_read+write per launch (8-head capture x5)",
-                     "algorithmic_bytes": int(attn_bytes)},
+        "roofline": roof,
         "gpu_launches": launches_per_step * args.steps,
+        "gpu_launches_note": f"{launches_per_step} library kernels per step; the planner leg and e2e are timed "
+                             "separately",
         "clocks": clocks,
         "e2e": e2e,
     }
@@ -330,16 +464,6 @@ def run_ours(args, rank, world, local_rank):
 
 
 # ------------------------------------------------------------------ Light-Ulysses share
-def attn_roofline(flops, ms, peaks, mode, d):
-    """The attention kernel against the dense 8-bit (2x sustained bf16) or bf16 peak."""
-    peak = (2.0 if mode == "int8fp8" else 1.0) * peaks["bf16_sustained"]
-    achieved = flops / (ms * 1e-3) / 1e12
-    return {"bound": "tensor", "kernel": f"sparse_attn_kernel<{d},{mode}>", "achieved": round(achieved, 1),
-            "peak": round(peak, 1), "unit": "TFLOP/s", "frac": round(achieved / peak, 3), "traffic": None,
-            "peak_note": f"{'2 x ' if mode == 'int8fp8' else ''}{peaks['source']} sustained bf16 "
-                         f"({peaks['bf16_sustained']})"}
-
-
 def ulysses_cpu_sample(N, B, H, d, L, flops, sample_tokens=256, attn=None):
     """The oracle on a bounded sample of one rank's share: the exchange steps
     (pack/unpack of the Q/K/V payload and of the output) on `sample_tokens` of
@@ -448,7 +572,7 @@ def run_ulysses_share(args):
             "data": "synthetic N(0,1) shards", "config": {"workload": f"{args.workload} B={B} H={H} d={d} L={L} N={N}",
                                                           "shard_tokens": Lr, "heads_after_exchange": Hr},
             "breakdown_ms": {n: round(v, 4) for n, v in per.items()}, "phases": phases,
-            "roofline": attn_roofline(flops, per["attn"], peaks, args.mode, d),
+            "roofline": attn_roofline(flops, per["attn"], peaks, args.mode, d, (clocks or {}).get("sm_mhz")),
             "gpu_launches": (10 if args.mode == "int8fp8" else 8) * args.steps, "clocks": clocks, "e2e": None,
             "cpu_baseline": (None if args.no_cpu_baseline else ulysses_cpu_sample(N, B, H, d, L, flops)),
             "note": "the all-to-all is not timed (one GPU); the send buffer stands in for the received one"}
@@ -632,6 +756,9 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--e2e-heads-per-chunk", type=int, default=2)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--planner-steps", type=int, default=10, help="timed calls of the planner alone")
+    ap.add_argument("--peaks", action="store_true",
+                    help="measure the dense int8 and fp8 GEMM peaks (cuBLAS) and print them as JSON")
     ap.add_argument("--heads", type=int, default=0, help="fewer heads: a smaller case for profiling only")
     ap.add_argument("--workload", default=WORKLOAD, choices=["480p", "720p", "long"],
                     help="grid shape (the headline is 720p; the others are characterisation runs)")
@@ -649,6 +776,9 @@ def main():
     ap.add_argument("--gemm-n", type=int, default=0, help="--gemm with another output width (characterisation)")
     ap.add_argument("--gemm-k", type=int, default=0, help="--gemm with another input width (characterisation)")
     args = ap.parse_args()
+    if args.peaks:
+        print(json.dumps(measure_8bit_peaks()))
+        return
     if args.gemm:
         print(json.dumps(run_nvfp4_gemm(args)))
         return

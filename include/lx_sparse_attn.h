@@ -243,9 +243,11 @@ lx_status lx_quantize_v(const lx_bhld* V, uint8_t* vc, float* vs, uint32_t* amax
  *
  * First-call setup: the first call on each device looks up the array's device
  * address (cudaGetSymbolAddress, with that device current, guarded by a host
- * mutex) and caches it; later calls only read the cache.  That lookup may load
- * the library's device code, so make the first call on a device before any
- * stream capture begins.
+ * mutex) and caches it together with the device's current context; later
+ * calls in the same context only read the cache.  After a cudaDeviceReset the
+ * device has a new context, and the next call looks the address up again.
+ * The lookup may load the library's device code, so make the first call on a
+ * device (and the first after a reset) before any stream capture begins.
  *
  * Errors: LX_ERR_WORKSPACE when B*H*D > LX_NOALLOC_AMAX_MAX (nothing is
  * launched); LX_ERR_CUDA when the lookup fails; otherwise as lx_quantize_v. */

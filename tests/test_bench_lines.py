@@ -3,16 +3,47 @@ roofline object and the oracle CPU baseline of a Light-Ulysses rank share."""
 import bench
 
 
-PEAKS = {"hbm_gbs": 6548.8, "bf16": 1628.7, "bf16_sustained": 1380.3, "source": "measured"}
+PEAKS = {"hbm_gbs": 6548.8, "bf16": 1628.7, "bf16_sustained": 1380.3, "source": "measured",
+         "int8": 3000.0, "fp8": 3400.0, "int8_sustained": 2600.0, "fp8_sustained": 2900.0,
+         "source_8bit": "measured"}
 
 
 def test_attn_roofline_int8_and_bf16():
     r = bench.attn_roofline(2.0e12, 2.0, PEAKS, "int8fp8", 128)      # 1000 TFLOP/s
     assert r["bound"] == "tensor" and r["unit"] == "TFLOP/s"
-    assert r["achieved"] == 1000.0 and r["peak"] == 2760.6
-    assert r["frac"] == round(1000.0 / 2760.6, 3)
+    # the 8-bit burst peak is the larger of the measured int8 and fp8 figures
+    assert r["achieved"] == 1000.0 and r["peak"] == 3400.0
+    assert r["frac"] == round(1000.0 / 3400.0, 3)
+    assert r["frac_of_sustained"] == round(1000.0 / 2900.0, 3)
+    assert "tcgen05_peak_at_clock" not in r
     b = bench.attn_roofline(2.0e12, 2.0, PEAKS, "bf16", 128)
-    assert b["peak"] == 1380.3 and b["kernel"] == "sparse_attn_kernel<128,bf16>"
+    assert b["peak"] == 1628.7 and b["kernel"] == "sparse_attn_kernel<128,bf16>"
+    assert b["frac_of_sustained"] == round(1000.0 / 1380.3, 3)
+
+
+def test_attn_roofline_tcgen05_rate_at_the_sampled_clock():
+    # 8192 MAC/clk/SM x 2 x 148 SMs x 1965 MHz = 4764.9 TFLOP/s for 8-bit, half for bf16
+    r = bench.attn_roofline(2.0e12, 2.0, PEAKS, "int8fp8", 128, sm_mhz=1965.0)
+    assert r["tcgen05_peak_at_clock"] == round(2 * 8192 * 148 * 1965e6 / 1e12, 1)
+    assert r["frac_of_tcgen05_at_clock"] == round(1000.0 / (2 * 8192 * 148 * 1965e6 / 1e12), 3)
+    b = bench.attn_roofline(2.0e12, 2.0, PEAKS, "bf16", 128, sm_mhz=1965.0)
+    assert b["tcgen05_peak_at_clock"] == round(8192 * 148 * 1965e6 / 1e12, 1)
+
+
+def test_peaks_without_8bit_file_fall_back_to_twice_bf16_burst(tmp_path, monkeypatch):
+    monkeypatch.setattr(bench, "PEAKS_8BIT", str(tmp_path / "absent.json"))
+    p = bench._peaks()
+    assert p["int8"] == p["fp8"] == 2.0 * p["bf16"]
+    assert p["int8_sustained"] == 2.0 * p["bf16_sustained"]
+
+
+def test_attn_traffic_is_keyed_by_kernel_source(monkeypatch):
+    import hashlib
+    h = hashlib.sha256(open(bench.ATTN_SRC, "rb").read()).hexdigest()
+    monkeypatch.setattr(bench, "ATTN_DRAM_BYTES", {"0" * 64: (1, "stale")})
+    assert bench.attn_traffic()[0] is None
+    monkeypatch.setattr(bench, "ATTN_DRAM_BYTES", {h: (123, "capture")})
+    assert bench.attn_traffic() == (123, "capture")
 
 
 def test_ulysses_cpu_sample_combines_exchange_and_attention():

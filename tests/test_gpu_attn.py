@@ -153,3 +153,29 @@ def test_one_call_equals_plan_then_forward(mode):
     assert lx.lx_last_device_status() == 0
     assert torch.equal(plan.idx, plan2.idx) and torch.equal(plan.mask, plan2.mask)
     assert torch.equal(O1, O2)
+
+
+@pytest.mark.parametrize("mode", ["int8fp8", "bf16"])
+def test_attn_720p_whole_head(mode):
+    """Every query block of one head at the 720p grid (1182 blocks, the ragged
+    last one included), element by element, in the launch the benchmark times
+    (all 40 heads in one call)."""
+    w = synth.WORKLOADS["720p"]
+    Q, K, V = synth.make_qkv(w.B, w.H, w.d, w.grid, seed=0, device=DEV)
+    plan = lx.lx_sparse_attn_plan(Q, K, w.keep)
+    O = lx.lx_sparse_attn_fwd(Q, K, V, plan, mode)
+    assert lx.lx_last_device_status() == 0
+    h = 23
+    Qh, Kh, Vh = (x[:, h:h + 1].cpu() for x in (Q, K, V))
+    idx = to_np(plan.idx)[:, h:h + 1]
+    Oh = O[:, h:h + 1]
+    del Q, K, V
+    blocks = _all_blocks(1, 1, w.L)
+    if mode == "bf16":
+        R = oracle.attn_ref_exact(Qh, Kh, Vh, idx)
+        mx, _ = compare_rows(Oh, R, w.L, blocks)
+        assert mx <= TOL_BF16_MAXABS, mx
+    else:
+        R = oracle.attn_ref_int8fp8(Qh, Kh, Vh, idx)
+        mx, rl1 = compare_rows(Oh, R, w.L, blocks)
+        assert mx <= TOL_I8_MAXABS and rl1 <= TOL_I8_RELL1, (mx, rl1)

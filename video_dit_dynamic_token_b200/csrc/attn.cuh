@@ -6,25 +6,30 @@
 // 720p Video in 3.8s", §3 Dynamic sparse attention: the same in English.
 //
 // Tile: one CTA owns two adjacent 64-row query blocks (2p, 2p+1), run as two
-// independent M=64 streams A and B in lockstep.  Step c computes query block
-// 2p against its c-th kept key block and query block 2p+1 against ITS c-th
-// kept key block, so every row works on one of its own kept blocks at every
-// step and a CTA takes exactly k steps (no union of the two lists, no idle
-// rows).  The two M=64 accumulators of a step share TMEM columns: stream A in
-// lanes 0-15 and stream B in lanes 16-31 of each 32-lane subpartition (the
-// half-subpartition layout of an M=64 tcgen05 accumulator), so one warp's
-// 32x32b TMEM load returns 16 rows of A and 16 rows of B.
+// independent M=64 streams A and B in lockstep; two CTAs share an SM.  Step c
+// computes query block 2p against its c-th kept key block and query block
+// 2p+1 against ITS c-th kept key block, so every row works on one of its own
+// kept blocks at every step and a CTA takes exactly k steps (no union of the
+// two lists, no idle rows).  The two M=64 accumulators of a step share TMEM
+// columns: stream A in lanes 0-15 and stream B in lanes 16-31 of each 32-lane
+// subpartition (the half-subpartition layout of an M=64 tcgen05
+// accumulator), so one warp's 32x32b TMEM load returns 16 rows of A and 16
+// rows of B, and each softmax thread owns a whole row of S and of O.
 //
-// S is computed for two consecutive kept blocks of a stream at once (M=64,
-// N=128 over the stacked blocks); P.V and the O rescale stay per 64-key block.
+// Pipeline (per step c, every buffer two-deep by step parity): K and V blocks
+// of both streams in two-stage rings, S(c) (M=64, N=64) in TMEM columns
+// [64 (c & 1), +64), P(c) in shared memory.  S(c+2) is issued as soon as the
+// softmax has read S(c), early in step c, and its K blocks load while S(c)
+// computes; P.V(c) is issued when P(c) is written.  The softmax waits for
+// P.V(c-1) only when one of its warp's rows must rescale O.
 //
-// Roles (6 warps): warp 0 = TMA producer (Q once; K blocks of both streams, a
-// pair of steps at a time, into one stage; V blocks into a 2-stage ring);
+// Roles (6 warps): warp 0 = TMA producer (Q once, then K and V blocks);
 // warp 1 = TMEM allocator + MMA issuer (S_A, S_B = Q K^T into the S columns,
 // then O_A, O_B += P V into the O columns, P and V read from shared memory);
-// warps 2..5 = softmax /
-// correction / epilogue, one thread per (stream, row): thread t of warp w
-// reads TMEM lane 32*(w%4) + t, i.e. row 16*(w%4) + t%16 of stream t/16.
+// both run their loops warp-wide and issue from one elected lane.  Warps
+// 2..5 = softmax / correction / epilogue, one thread per (stream, row): thread
+// t of warp w reads TMEM lane 32*(w%4) + t, i.e. row 16*(w%4) + t%16 of stream
+// t/16.
 //
 // INT8/FP8 mode follows the P-quantisation protocol: per 64-key block c the
 // row max becomes m_c = max(m_{c-1}, max S_c); P~ = E4M3(448 exp(S_c - m_c));
@@ -47,23 +52,24 @@ struct AttnCfg {
   static constexpr int NATOM = ROWB / ATOM;               // atom columns per row
   static constexpr int Q_BYTES = 128 * ROWB;              // rows 0-63: stream A, rows 64-127: stream B
   static constexpr int KV_BYTES = 64 * ROWB;              // one K (or V) block
-  static constexpr int KPAIR_BYTES = 2 * KV_BYTES;        // one stream's two K blocks: [NATOM][128 rows][ATOM]
-  static constexpr int VSTAGE = 2;                        // V ring (A and B blocks per stage)
+  static constexpr int STAGE_BYTES = 2 * KV_BYTES;        // one step's blocks of both streams: [stream][NATOM][64][ATOM]
+  static constexpr int VSTAGE = 2;                        // K and V rings of two steps each
   static constexpr int P_ROWB = 64 * ESZ;                 // P row: 64 keys
   static constexpr int P_BYTES = 64 * P_ROWB;             // P of one stream, K-major, swizzled
   static constexpr uint32_t SW_QKV = ATOM == 128 ? SW_128B : SW_64B;
   static constexpr uint32_t SW_P = P_ROWB == 128 ? SW_128B : SW_64B;
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_K = OFF_Q + Q_BYTES;
-  static constexpr int OFF_V = OFF_K + 2 * KPAIR_BYTES;
+  static constexpr int OFF_V = OFF_K + 2 * STAGE_BYTES;
   static constexpr int OFF_P = OFF_V + VSTAGE * 2 * KV_BYTES;
-  static constexpr int OFF_IDX = OFF_P + 2 * P_BYTES;     // the two kept lists (2 x k int32) follow
-  static constexpr int S_COL = 0;                         // TMEM: S of a step pair, cols [0, 128)
+  static constexpr int OFF_IDX = OFF_P + 4 * P_BYTES;     // P: [step parity][stream]; then the two kept
+                                                          // lists (2 x k int32) and their K scales (2 x k fp32)
+  static constexpr int S_COL = 0;                         // TMEM: S of step c in columns [64 (c & 1), +64)
   static constexpr int O_COL = 128;                       // TMEM: O accumulator, D cols
   static constexpr uint32_t LANE_B = 16u << 16;           // TMEM address offset of stream B (lane 16)
   static constexpr uint32_t TMEM_COLS = 256;
   static constexpr uint32_t IDESC_S =
-      instr_desc(I8 ? IDESC_DS32 : IDESC_DF32, I8 ? IDESC_S8 : IDESC_BF16, I8 ? IDESC_S8 : IDESC_BF16, 0, 0, 64, 128);
+      instr_desc(I8 ? IDESC_DS32 : IDESC_DF32, I8 ? IDESC_S8 : IDESC_BF16, I8 ? IDESC_S8 : IDESC_BF16, 0, 0, 64, 64);
   static constexpr uint32_t IDESC_PV =
       instr_desc(IDESC_DF32, I8 ? IDESC_E4M3 : IDESC_BF16, I8 ? IDESC_E4M3 : IDESC_BF16, 0, 1, 64, D);
   static constexpr int KEYS_PER_MMA = 32 / ESZ;           // 32 bytes of K per instruction
@@ -94,6 +100,12 @@ constexpr uint32_t kMagicBits = 0x4B400000u;
 constexpr float kMagic = 12582912.0f;
 constexpr float kLog2_448 = 8.807354922057604f;
 
+// A bounded wait taken by a whole warp; the verdict is made warp-uniform.
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, const volatile int* abort,
+                                          uint64_t limit_ns) {
+  return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort, limit_ns));
+}
+
 template <int D, bool I8>
 __global__ void __launch_bounds__(192, I8 ? 2 : 1)
     sparse_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
@@ -101,8 +113,12 @@ __global__ void __launch_bounds__(192, I8 ? 2 : 1)
   using C = AttnCfg<D, I8>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  __shared__ uint64_t bar_q, bar_kfull, bar_kempty, bar_vfull[C::VSTAGE],
-      bar_vempty[C::VSTAGE], bar_sfull, bar_sfree, bar_pfull, bar_odone, bar_drain;
+  // per step parity b: kfull/vfull[b] the K/V blocks have landed; sfull[b]
+  // S is complete (its K stage is free again); sfree[b] the softmax has read
+  // S; pfull[b] P is written; odone[b] P.V is complete (its V stage and P
+  // tiles are free)
+  __shared__ uint64_t bar_q, bar_kfull[2], bar_vfull[2], bar_sfull[2], bar_sfree[2], bar_pfull[2], bar_odone[2],
+      bar_drain;
   __shared__ uint32_t tmem_slot;
   __shared__ volatile int abort_flag;
   __shared__ int never_abort;
@@ -114,23 +130,22 @@ __global__ void __launch_bounds__(192, I8 ? 2 : 1)
   const int qb0 = 2 * pair, qb1 = 2 * pair + 1;
   const bool has1 = qb1 < prm.nB;
   const int n = prm.k;  // steps: every stream walks exactly k kept blocks
-  const int npairs = (n + 1) >> 1;  // S is computed for steps 2p and 2p+1 together
   int32_t* idx0 = reinterpret_cast<int32_t*>(sm + C::OFF_IDX);
   int32_t* idx1 = idx0 + n;
+  float* skl0 = reinterpret_cast<float*>(idx1 + n);   // K scale of each kept block (INT8/FP8)
+  float* skl1 = skl0 + n;
 
   // ---- prologue: barriers, the two kept lists (validated), TMEM
   if (threadIdx.x == 0) {
     mbar_init(&bar_q, 1);
-    mbar_init(&bar_kfull, 1);
-    mbar_init(&bar_kempty, 1);
-    for (int s = 0; s < C::VSTAGE; ++s) {
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&bar_kfull[s], 1);
       mbar_init(&bar_vfull[s], 1);
-      mbar_init(&bar_vempty[s], 1);
+      mbar_init(&bar_sfull[s], 1);
+      mbar_init(&bar_sfree[s], 128);   // every softmax thread arrives
+      mbar_init(&bar_pfull[s], 128);
+      mbar_init(&bar_odone[s], 1);
     }
-    mbar_init(&bar_sfull, 1);
-    mbar_init(&bar_sfree, 128);
-    mbar_init(&bar_pfull, 128);
-    mbar_init(&bar_odone, 1);
     mbar_init(&bar_drain, 1);
     abort_flag = 0;
     never_abort = 0;
@@ -148,6 +163,10 @@ __global__ void __launch_bounds__(192, I8 ? 2 : 1)
       if (j1 < 0 || j1 >= prm.nB || (t > 0 && r1[t - 1] >= j1)) bad = true;
       idx0[t] = (j0 < 0 || j0 >= prm.nB) ? 0 : j0;
       idx1[t] = (j1 < 0 || j1 >= prm.nB) ? 0 : j1;
+      if constexpr (I8) {
+        skl0[t] = prm.sk[bh * prm.nB + idx0[t]];
+        skl1[t] = prm.sk[bh * prm.nB + idx1[t]];
+      }
     }
     if (bad) report_error(-7);
   }
@@ -162,81 +181,84 @@ __global__ void __launch_bounds__(192, I8 ? 2 : 1)
   const uint32_t sQ = smem_u32(sm + C::OFF_Q);
 
   if (warp == 0) {
-    // ================= TMA producer =================
-    if (lane == 0) {
+    // ================= TMA producer (warp-wide loop, one elected lane issues) =================
+    // Order K(0), K(1), V(0), then K(c+2), V(c+1) for c = 0, 1, ...: K(c)
+    // reuses the stage of K(c-2) once S(c-2) is complete, V(c) that of V(c-2)
+    // once P.V(c-2) is; S(c) is issued about two steps before P.V(c), so K
+    // runs ahead of V.
+    const bool leader = elect_one();
+    if (leader) {
       prefetch_tensormap(&tmQ);
       prefetch_tensormap(&tmK);
       prefetch_tensormap(&tmV);
       mbar_arrive_expect_tx(&bar_q, C::Q_BYTES);
       for (int a = 0; a < C::NATOM; ++a)
         tma_load_4d(sm + C::OFF_Q + a * 128 * C::ATOM, &tmQ, &bar_q, a * C::ATOM / C::ESZ, qb0 * kBlock, h_idx, b_idx);
-      const uint32_t kv_tx = (has1 ? 2 : 1) * C::KV_BYTES;
-      bool ok = true;
-      int nk = 0, nv = 0;  // K pairs and V steps issued so far
-      for (int c = 0; c < n; ++c) {
-        if ((c & 1) == 0) {
-          // K blocks of steps c and c+1 (both streams) into the pair stage,
-          // once S of the previous pair has read it
-          const int p = c >> 1;
-          ok = p == 0 || mbar_wait(&bar_kempty, (p - 1) & 1, &abort_flag, prm.limit_ns);
-          if (!ok) break;
-          const int nb = (c + 1 < n) ? 2 : 1;
-          mbar_arrive_expect_tx(&bar_kfull, (uint32_t)nb * kv_tx);
-          for (int s = 0; s < (has1 ? 2 : 1); ++s) {
-            const int32_t* ids = s ? idx1 : idx0;
-            for (int b = 0; b < nb; ++b)
-              for (int a = 0; a < C::NATOM; ++a)
-                tma_load_4d(sm + C::OFF_K + s * C::KPAIR_BYTES + a * 128 * C::ATOM + b * 64 * C::ATOM, &tmK,
-                            &bar_kfull, a * C::ATOM / C::ESZ, ids[c + b] * kBlock, h_idx, b_idx);
-          }
-          ++nk;
-        }
-        const int vs = c % C::VSTAGE;
-        ok = c < C::VSTAGE || mbar_wait(&bar_vempty[vs], ((c / C::VSTAGE) - 1) & 1, &abort_flag, prm.limit_ns);
-        if (!ok) break;
-        const int j0 = idx0[c], j1 = idx1[c];
-        uint8_t* sv = sm + C::OFF_V + vs * 2 * C::KV_BYTES;
-        mbar_arrive_expect_tx(&bar_vfull[vs], kv_tx);
-        for (int a = 0; a < C::NATOM; ++a) {
-          tma_load_4d(sv + a * 64 * C::ATOM, &tmV, &bar_vfull[vs], a * C::ATOM / C::ESZ, j0 * kBlock, h_idx, b_idx);
-          if (has1)
-            tma_load_4d(sv + C::KV_BYTES + a * 64 * C::ATOM, &tmV, &bar_vfull[vs], a * C::ATOM / C::ESZ,
-                        j1 * kBlock, h_idx, b_idx);
-        }
-        ++nv;
-      }
-      if (!ok) {
-        abort_flag = 1;
-        report_error(-6);
-      }
-      // drain: every issued load lands before the CTA may exit
-      mbar_wait(&bar_q, 0, &never_abort, prm.limit_ns);
-      if (nk > 0) mbar_wait(&bar_kfull, (nk - 1) & 1, &never_abort, prm.limit_ns);
-      for (int cc = nv - C::VSTAGE < 0 ? 0 : nv - C::VSTAGE; cc < nv; ++cc)
-        mbar_wait(&bar_vfull[cc % C::VSTAGE], (cc / C::VSTAGE) & 1, &never_abort, prm.limit_ns);
     }
+    const uint32_t kv_tx = (has1 ? 2 : 1) * C::KV_BYTES;
+    bool ok = true;
+    int nk = 0, nv = 0;  // K and V steps issued
+    const int nsteps = 2 * n + 1;
+    for (int step = 0; ok && step < nsteps; ++step) {
+      // steps 0, 1, 2: K0 K1 V0; then K((s+1)/2) at odd s >= 3, V(s/2 - 1) at even s >= 4
+      const bool do_k = step < 2 || (step > 2 && (step & 1));
+      const int c = step < 2 ? step : (step == 2 ? 0 : (do_k ? (step + 1) >> 1 : (step >> 1) - 1));
+      if (c >= n) continue;
+      if (c >= 2) {
+        ok = warp_wait(do_k ? &bar_sfull[c & 1] : &bar_odone[c & 1], ((c >> 1) - 1) & 1, &abort_flag, prm.limit_ns);
+        if (!ok) break;
+      }
+      if (leader) {
+        uint64_t* full = do_k ? &bar_kfull[c & 1] : &bar_vfull[c & 1];
+        uint8_t* stage = sm + (do_k ? C::OFF_K : C::OFF_V) + (c & 1) * C::STAGE_BYTES;
+        const CUtensorMap* map = do_k ? &tmK : &tmV;
+        mbar_arrive_expect_tx(full, kv_tx);
+        for (int s = 0; s < (has1 ? 2 : 1); ++s) {
+          const int j = (s ? idx1 : idx0)[c];
+          for (int a = 0; a < C::NATOM; ++a)
+            tma_load_4d(stage + s * C::KV_BYTES + a * 64 * C::ATOM, map, full, a * C::ATOM / C::ESZ, j * kBlock,
+                        h_idx, b_idx);
+        }
+      }
+      __syncwarp();
+      if (do_k) ++nk;
+      else ++nv;
+    }
+    if (!ok && leader) {
+      abort_flag = 1;
+      report_error(-6);
+    }
+    // drain: every issued load lands before the CTA may exit
+    if (leader) {
+      mbar_wait(&bar_q, 0, &never_abort, prm.limit_ns);
+      for (int c = nk - 2 < 0 ? 0 : nk - 2; c < nk; ++c)
+        mbar_wait(&bar_kfull[c & 1], (c >> 1) & 1, &never_abort, prm.limit_ns);
+      for (int c = nv - 2 < 0 ? 0 : nv - 2; c < nv; ++c)
+        mbar_wait(&bar_vfull[c & 1], (c >> 1) & 1, &never_abort, prm.limit_ns);
+    }
+    __syncwarp();
   } else if (warp == 1) {
-    // ================= MMA issuer =================
-    if (lane == 0) {
-      // Descriptors of stage 0 / stream A; a shared-memory descriptor's start
-      // address sits in its low 14 bits (address >> 4, below 256 KB), so other
-      // stages, streams and K steps are plain additions of (offset >> 4).
-      const uint64_t dQ = smem_desc(sQ, 16, 8 * C::ATOM, C::SW_QKV);
-      const uint64_t dK = smem_desc(smem_u32(sm + C::OFF_K), 16, 8 * C::ATOM, C::SW_QKV);
-      const uint64_t dP = smem_desc(smem_u32(sm + C::OFF_P), 16, 8 * C::P_ROWB, C::SW_P);
-      const uint64_t dV = smem_desc(smem_u32(sm + C::OFF_V), 64 * C::ATOM, 8 * C::ATOM, C::SW_QKV);
-      bool ok = mbar_wait(&bar_q, 0, &abort_flag, prm.limit_ns);
-      tc_fence_after();
-      // Iteration c issues S of pair p+1 (when c = 2p+1; pair 0 goes first)
-      // and then P(c).V.  S of pair p+1 needs the softmax to have read both
-      // halves of pair p's S, which it does at the start of step 2p+1.
-      for (int c = -1; ok && c < n; ++c) {
-        const int p = (c + 1) >> 1;  // the pair whose S is issued in this iteration
-        if ((c & 1) != 0 && p < npairs) {  // c = -1, 1, 3, ...
-          ok = mbar_wait(&bar_kfull, p & 1, &abort_flag, prm.limit_ns) &&
-               mbar_wait(&bar_sfree, p & 1, &abort_flag, prm.limit_ns);
-          if (!ok) break;
-          tc_fence_after();
+    // ================= MMA issuer (warp-wide loop, one elected lane issues) =================
+    // Descriptors of stage 0 / stream A; a shared-memory descriptor's start
+    // address sits in its low 14 bits (address >> 4, below 256 KB), so other
+    // stages, streams and K steps are plain additions of (offset >> 4).
+    const uint64_t dQ = smem_desc(sQ, 16, 8 * C::ATOM, C::SW_QKV);
+    const uint64_t dK = smem_desc(smem_u32(sm + C::OFF_K), 16, 8 * C::ATOM, C::SW_QKV);
+    const uint64_t dP = smem_desc(smem_u32(sm + C::OFF_P), 16, 8 * C::P_ROWB, C::SW_P);
+    const uint64_t dV = smem_desc(smem_u32(sm + C::OFF_V), 64 * C::ATOM, 8 * C::ATOM, C::SW_QKV);
+    const bool leader = elect_one();
+    bool ok = warp_wait(&bar_q, 0, &abort_flag, prm.limit_ns);
+    tc_fence_after();
+    // S(0), S(1); then for each step c: S(c+2) once the softmax has read S(c)
+    // (early in step c) and P.V(c) once it has written P(c) (at its end)
+    for (int it = -2; ok && it < n; ++it) {
+      const int cs = it + 2;   // the step whose S is issued in this iteration
+      if (cs < n) {
+        ok = warp_wait(&bar_kfull[cs & 1], (cs >> 1) & 1, &abort_flag, prm.limit_ns) &&
+             warp_wait(&bar_sfree[cs & 1], (cs >> 1) & 1, &abort_flag, prm.limit_ns);
+        if (!ok) break;
+        tc_fence_after();
+        if (leader) {
 #pragma unroll
           for (int s = 0; s < 2; ++s) {
             if (s == 1 && !has1) break;
@@ -244,45 +266,52 @@ __global__ void __launch_bounds__(192, I8 ? 2 : 1)
             for (int kk = 0; kk < C::ROWB / 32; ++kk) {
               const int a = (kk * 32) / C::ATOM, off = (kk * 32) % C::ATOM;
               const uint64_t ad = dQ + (uint64_t)((a * 128 * C::ATOM + s * 64 * C::ATOM + off) >> 4);
-              const uint64_t bd = dK + (uint64_t)((s * C::KPAIR_BYTES + a * 128 * C::ATOM + off) >> 4);
+              const uint64_t bd =
+                  dK + (uint64_t)(((cs & 1) * C::STAGE_BYTES + s * C::KV_BYTES + a * 64 * C::ATOM + off) >> 4);
               // INT8: accumulate onto the magic-number start the softmax warps wrote
-              mma_ss<I8 ? KIND_I8 : KIND_F16>(tbase + s * C::LANE_B + C::S_COL, ad, bd, C::IDESC_S,
+              mma_ss<I8 ? KIND_I8 : KIND_F16>(tbase + s * C::LANE_B + C::S_COL + 64 * (cs & 1), ad, bd, C::IDESC_S,
                                               (I8 || kk > 0) ? 1u : 0u);
             }
           }
-          mma_commit(&bar_sfull);
-          mma_commit(&bar_kempty);
+          mma_commit(&bar_sfull[cs & 1]);
         }
-        if (c >= 0) {
-          const int vs = c % C::VSTAGE;
-          ok = mbar_wait(&bar_vfull[vs], (c / C::VSTAGE) & 1, &abort_flag, prm.limit_ns) &&
-               mbar_wait(&bar_pfull, c & 1, &abort_flag, prm.limit_ns);
-          if (!ok) break;
-          tc_fence_after();
-          const uint64_t dVs = dV + (uint64_t)((vs * 2 * C::KV_BYTES) >> 4);
+        __syncwarp();
+      }
+      const int c = it;        // the step whose P.V is issued in this iteration
+      if (c >= 0) {
+        ok = warp_wait(&bar_vfull[c & 1], (c >> 1) & 1, &abort_flag, prm.limit_ns) &&
+             warp_wait(&bar_pfull[c & 1], (c >> 1) & 1, &abort_flag, prm.limit_ns);
+        if (!ok) break;
+        tc_fence_after();
+        if (leader) {
+          const uint64_t dVs = dV + (uint64_t)(((c & 1) * C::STAGE_BYTES) >> 4);
+          const uint64_t dPc = dP + (uint64_t)(((c & 1) * 2 * C::P_BYTES) >> 4);
 #pragma unroll
           for (int s = 0; s < 2; ++s) {
             if (s == 1 && !has1) break;
 #pragma unroll
             for (int kk = 0; kk < 64 / C::KEYS_PER_MMA; ++kk) {
-              const uint64_t ad = dP + (uint64_t)((s * C::P_BYTES + kk * 32) >> 4);
+              const uint64_t ad = dPc + (uint64_t)((s * C::P_BYTES + kk * 32) >> 4);
               const uint64_t bd = dVs + (uint64_t)((s * C::KV_BYTES + kk * C::KEYS_PER_MMA * C::ATOM) >> 4);
               mma_ss<I8 ? KIND_F8F6F4 : KIND_F16>(tbase + s * C::LANE_B + C::O_COL, ad, bd, C::IDESC_PV,
                                                   (c > 0 || kk > 0) ? 1u : 0u);
             }
           }
-          mma_commit(&bar_odone);
-          mma_commit(&bar_vempty[vs]);
+          mma_commit(&bar_odone[c & 1]);
         }
+        __syncwarp();
       }
-      if (!ok) {
-        abort_flag = 1;
-        report_error(-6);
-      }
-      // drain: all issued MMAs complete before TMEM is released
+    }
+    if (!ok && leader) {
+      abort_flag = 1;
+      report_error(-6);
+    }
+    // drain: all issued MMAs complete before TMEM is released
+    if (leader) {
       mma_commit(&bar_drain);
       mbar_wait(&bar_drain, 0, &never_abort, prm.limit_ns);
     }
+    __syncwarp();
   } else {
     // ================= softmax / correction / epilogue =================
     const int quarter = warp & 3;
@@ -293,12 +322,10 @@ __global__ void __launch_bounds__(192, I8 ? 2 : 1)
     const int t = qblk * kBlock + row;            // token index of this row
     const uint32_t lane_addr = tbase + ((uint32_t)(quarter * 32) << 16);
     const int32_t* my_idx = stream ? idx1 : idx0;
-    const float* sk_row = prm.sk + bh * prm.nB;
+    const float* my_skl = stream ? skl1 : skl0;
     float sq = 1.0f;
     if constexpr (I8) sq = prm.sq[bh * prm.nB + min(qblk, prm.nB - 1)];
     float m_run = -INFINITY, l_run = 0.f;
-    // this thread's row of its stream's P tile (K-major, swizzled)
-    uint8_t* prow = sm + C::OFF_P + stream * C::P_BYTES;
     // the S columns start free (INT8: at the magic-number start value)
     if constexpr (I8) {
       uint32_t mg[32];
@@ -309,23 +336,16 @@ __global__ void __launch_bounds__(192, I8 ? 2 : 1)
       tmem_wait_st();
     }
     tc_fence_before();
-    mbar_arrive(&bar_sfree);
+    mbar_arrive(&bar_sfree[0]);
+    mbar_arrive(&bar_sfree[1]);
     bool ok = true;
-    int j_next = n > 0 ? my_idx[0] : 0;
-    float sk_next = (I8 && n > 0) ? __ldg(sk_row + j_next) : 1.f;
     for (int c = 0; c < n; ++c) {
-      const int j = j_next;
-      const float skj = sk_next;
-      if (c + 1 < n) {  // the next step's block and K scale, fetched a step ahead
-        j_next = my_idx[c + 1];
-        if constexpr (I8) sk_next = __ldg(sk_row + j_next);
-      }
-      const int half = c & 1;  // which 64 columns of the pair's S
+      const int j = my_idx[c];
+      const float skj = I8 ? my_skl[c] : 1.f;
+      const int half = c & 1;  // S buffer and P tiles of this step
       const uint32_t s_addr = lane_addr + C::S_COL + 64 * half;
-      if (half == 0) {
-        ok = mbar_wait(&bar_sfull, (c >> 1) & 1, &abort_flag, prm.limit_ns);
-        if (!ok) break;
-      }
+      ok = warp_wait(&bar_sfull[half], (c >> 1) & 1, &abort_flag, prm.limit_ns);
+      if (!ok) break;
       tc_fence_after();
       uint32_t sv[64];
       {
@@ -335,9 +355,8 @@ __global__ void __launch_bounds__(192, I8 ? 2 : 1)
         tmem_ld32(s_addr + 32, hi);
         tmem_wait_ld();
       }
-      // INT8: restart these columns at the magic value; after the second half
-      // of the pair the S columns go back to the MMA thread at once, so the
-      // next pair's S = QK^T runs while this block's softmax runs
+      // INT8: restart these columns at the magic value, then hand the S
+      // buffer back to the MMA warp: S(c+2) runs while this step's softmax runs
       if constexpr (I8) {
         uint32_t mg[32];
 #pragma unroll
@@ -346,10 +365,8 @@ __global__ void __launch_bounds__(192, I8 ? 2 : 1)
         tmem_st32(s_addr + 32, mg);
         tmem_wait_st();
       }
-      if (half == 1) {
-        tc_fence_before();
-        mbar_arrive(&bar_sfree);
-      }
+      tc_fence_before();
+      mbar_arrive(&bar_sfree[half]);
       const int nvalid = (j == prm.nB - 1) ? (prm.L - j * kBlock) : kBlock;
       float sc = prm.scale_log2;
       if constexpr (I8) sc *= sq * skj;
@@ -423,14 +440,19 @@ __global__ void __launch_bounds__(192, I8 ? 2 : 1)
 #pragma unroll
         for (int i = 0; i < PW; ++i) pk[i] = 0u;
       }
-      if (c >= 1) {
-        // the previous block's P.V is complete: O may be rescaled and the P
-        // tiles may be overwritten
-        ok = mbar_wait(&bar_odone, (c - 1) & 1, &abort_flag, prm.limit_ns);
+      // P tiles of parity c & 1 are free once P.V(c-2) is complete
+      if (c >= 2) {
+        ok = warp_wait(&bar_odone[half], ((c - 2) >> 1) & 1, &abort_flag, prm.limit_ns);
         if (!ok) break;
-        tc_fence_after();
+      }
+      if (c >= 1) {
+        // a rescale of O needs the previous block's P.V complete; a warp none
+        // of whose rows needs one does not wait for it
         const bool need_rescale = valid && m_run != -INFINITY && m_new > m_run;
         if (__any_sync(0xffffffffu, need_rescale)) {
+          ok = warp_wait(&bar_odone[(c - 1) & 1], ((c - 1) >> 1) & 1, &abort_flag, prm.limit_ns);
+          if (!ok) break;
+          tc_fence_after();
           const float f = need_rescale ? alpha : 1.f;
           const uint64_t f2 = f2pack(f, f);
 #pragma unroll
@@ -451,13 +473,14 @@ __global__ void __launch_bounds__(192, I8 ? 2 : 1)
         }
       }
       // P row into shared memory: the A operand of this stream's P.V
+      uint8_t* prow = sm + C::OFF_P + (half * 2 + stream) * C::P_BYTES;
 #pragma unroll
       for (int ch = 0; ch < C::P_ROWB / 16; ++ch)
         *reinterpret_cast<uint4*>(prow + swz_offset(row, ch, C::P_ROWB)) =
             make_uint4(pk[4 * ch], pk[4 * ch + 1], pk[4 * ch + 2], pk[4 * ch + 3]);
       fence_proxy_async_smem();
       tc_fence_before();
-      mbar_arrive(&bar_pfull);
+      mbar_arrive(&bar_pfull[half]);
       if (valid) {
         l_run = l_run * alpha + psum;
         m_run = m_new;
@@ -468,7 +491,7 @@ __global__ void __launch_bounds__(192, I8 ? 2 : 1)
       report_error(-6);
     } else {
       // epilogue: wait for the last P.V, normalise, store bf16 rows
-      ok = n == 0 || mbar_wait(&bar_odone, (n - 1) & 1, &abort_flag, prm.limit_ns);
+      ok = n == 0 || warp_wait(&bar_odone[(n - 1) & 1], ((n - 1) >> 1) & 1, &abort_flag, prm.limit_ns);
       if (!ok) {
         abort_flag = 1;
         report_error(-6);

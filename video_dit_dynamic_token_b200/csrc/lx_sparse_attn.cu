@@ -194,7 +194,8 @@ lx_status launch_attn(const CUtensorMap& mq, const CUtensorMap& mk, const CUtens
                       const lx_bhld* O, const float* qs, const float* ks, const float* vs, cudaStream_t s) {
   using C = lx::AttnCfg<D, I8>;
   const int64_t nB = plan->nB;
-  const size_t smem = 1024 + C::OFF_IDX + 2 * sizeof(int32_t) * (size_t)plan->k;
+  // the two kept lists and their K scales follow the tiles
+  const size_t smem = 1024 + C::OFF_IDX + 16 * (size_t)plan->k;
   if (smem > 227 * 1024) return LX_ERR_UNSUPPORTED;
   if (cudaFuncSetAttribute(lx::sparse_attn_kernel<D, I8>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
       cudaSuccess)
@@ -214,6 +215,7 @@ lx_status launch_attn(const CUtensorMap& mq, const CUtensorMap& mk, const CUtens
   p.sv = vs;
   p.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)D));
   p.limit_ns = kWaitLimitNs;
+  // one CTA per (pair of query blocks, b*h), head-major so that a head's K/V stays in L2
   dim3 grid((unsigned)((nB + 1) / 2), (unsigned)(plan->B * plan->H));
   lx::sparse_attn_kernel<D, I8><<<grid, 192, smem, s>>>(mq, mk, mv, p);
   return launch_status();
@@ -546,20 +548,49 @@ static __device__ __align__(256) uint32_t g_noalloc_amax[LX_NOALLOC_AMAX_MAX];
 namespace {
 constexpr int kMaxDevices = 64;
 std::mutex g_noalloc_mu;
-uint32_t* g_noalloc_ptr[kMaxDevices] = {};
+// Per device: the context the address was looked up in, and the address.  A
+// device reset gives the device a new primary context whose copy of the array
+// may sit elsewhere, so a cached address is reused only in the same context.
+struct NoallocEntry {
+  CUcontext ctx;
+  uint32_t* ptr;
+};
+NoallocEntry g_noalloc[kMaxDevices] = {};
 
-// Device address of g_noalloc_amax on the current device, looked up once.
+typedef CUresult (*CtxGetCurrentFn)(CUcontext*);
+CtxGetCurrentFn ctx_get_current_fn() {
+  static CtxGetCurrentFn fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<CtxGetCurrentFn>(p);
+  }
+  return fn;
+}
+
+// Device address of g_noalloc_amax on the current device, looked up once per
+// (device, context).
 lx_status noalloc_scratch(uint32_t** out) {
   int dev = -1;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) return LX_ERR_CUDA;
   if (dev >= kMaxDevices) return LX_ERR_UNSUPPORTED;
+  CtxGetCurrentFn get_ctx = ctx_get_current_fn();
+  if (!get_ctx) return LX_ERR_CUDA;
   std::lock_guard<std::mutex> lock(g_noalloc_mu);
-  if (!g_noalloc_ptr[dev]) {
+  NoallocEntry& e = g_noalloc[dev];
+  CUcontext ctx = nullptr;
+  if (get_ctx(&ctx) != CUDA_SUCCESS) return LX_ERR_CUDA;
+  if (!e.ptr || !ctx || e.ctx != ctx) {
+    // the lookup also makes the runtime's context current when none is yet
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_noalloc_amax) != cudaSuccess || !p) return LX_ERR_CUDA;
-    g_noalloc_ptr[dev] = static_cast<uint32_t*>(p);
+    if (get_ctx(&ctx) != CUDA_SUCCESS || !ctx) return LX_ERR_CUDA;
+    e.ctx = ctx;
+    e.ptr = static_cast<uint32_t*>(p);
   }
-  *out = g_noalloc_ptr[dev];
+  *out = e.ptr;
   return LX_OK;
 }
 }  // namespace
