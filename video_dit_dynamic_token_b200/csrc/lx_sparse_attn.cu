@@ -137,10 +137,10 @@ lx_status launch_qk_pass(const lx_bhld* Q, const lx_bhld* K, float* mq, float* m
   return launch_status();
 }
 
+// Scores of BH heads: tf32 x3 tensor-core GEMM, one 128 x 128 tile per CTA;
+// mq, mk, scores point at the first of the BH heads.
 template <int D>
-lx_status launch_score(const float* mq, const float* mk, int64_t BH, int64_t nB, int64_t k, float* scores,
-                       lx_plan* plan, cudaStream_t s) {
-  // scores: tf32 x3 tensor-core GEMM, one 128 x 128 tile per CTA
+lx_status launch_score_gemm(const float* mq, const float* mk, int64_t BH, int64_t nB, float* scores, cudaStream_t s) {
   CUtensorMap tq, tk;
   const auto f32 = CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
   if (!make_map(&tq, mq, f32, 4, 1, BH, nB, D, BH * nB * D, nB * D, D, lx::kSgK, lx::kSgM) ||
@@ -153,8 +153,14 @@ lx_status launch_score(const float* mq, const float* mk, int64_t BH, int64_t nB,
   dim3 ggrid((unsigned)((nB + lx::kSgM - 1) / lx::kSgM), (unsigned)((nB + lx::kSgN - 1) / lx::kSgN), (unsigned)BH);
   const int ldS = (int)score_ld(nB);
   lx::score_gemm_kernel<D><<<ggrid, 128, gsmem, s>>>(tq, tk, scores, (int)nB, ldS, kWaitLimitNs);
-  if (cudaGetLastError() != cudaSuccess) return LX_ERR_CUDA;
-  // selection: 8 rows per CTA, one warp per row
+  return launch_status();
+}
+
+// Top-k selection of BH heads: 8 score rows per CTA, one warp per row; the
+// pointers are those of the first of the BH heads (mask may be NULL).
+lx_status launch_select(const float* scores, int64_t BH, int64_t nB, int64_t k, int32_t* idx, uint32_t* mask,
+                        cudaStream_t s) {
+  const int ldS = (int)score_ld(nB);
   const size_t smem = sizeof(float) * ((size_t)lx::kScoreRows * ldS +
                                        lx::kScoreWarps * (lx::kBuckets + 2 * lx::kCandCap + ldS / 32));
   if (smem > 227 * 1024) return LX_ERR_UNSUPPORTED;
@@ -162,9 +168,17 @@ lx_status launch_score(const float* mq, const float* mk, int64_t BH, int64_t nB,
       cudaSuccess)
     return LX_ERR_CUDA;
   dim3 grid((unsigned)((nB + lx::kScoreRows - 1) / lx::kScoreRows), (unsigned)BH);
-  lx::select_topk_kernel<<<grid, 32 * lx::kScoreWarps, smem, s>>>(scores, (int)nB, (int)k, plan->idx, plan->mask,
-                                                                   ldS, kWaitLimitNs);
+  lx::select_topk_kernel<<<grid, 32 * lx::kScoreWarps, smem, s>>>(scores, (int)nB, (int)k, idx, mask, ldS,
+                                                                   kWaitLimitNs);
   return launch_status();
+}
+
+template <int D>
+lx_status launch_score(const float* mq, const float* mk, int64_t BH, int64_t nB, int64_t k, float* scores,
+                       lx_plan* plan, cudaStream_t s) {
+  lx_status st = launch_score_gemm<D>(mq, mk, BH, nB, scores, s);
+  if (st != LX_OK) return st;
+  return launch_select(scores, BH, nB, k, plan->idx, plan->mask, s);
 }
 
 template <int D, bool MEANS>

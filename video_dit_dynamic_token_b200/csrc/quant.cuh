@@ -124,7 +124,8 @@ __global__ void __launch_bounds__(128) qk_block_pass_kernel(BhldView q, BhldView
     // table part (0 t, 1 h, 2 w), base and pairs per position
     const float4* wrow = reinterpret_cast<const float4*>((isk ? pro.wk : pro.wq) + h * D + c * 8);
     const float4 w0 = __ldg(wrow), w1 = __ldg(wrow + 1);
-    const float wv[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+    // weights of this thread's 4 channel pairs, packed for f32x2 arithmetic
+    const uint64_t wp[4] = {f2pack(w0.x, w0.y), f2pack(w0.z, w0.w), f2pack(w1.x, w1.y), f2pack(w1.z, w1.w)};
     int pax[4], pbase[4], pstride[4];
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
@@ -161,32 +162,37 @@ __global__ void __launch_bounds__(128) qk_block_pass_kernel(BhldView q, BhldView
         }
       }
       const int row = r + RG * i;
+      // the row's 8 channels as 4 packed (even, odd) pairs
       const uint32_t wd[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
-      float x[8];
+      uint64_t x2[4];
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        x[2 * e] = bf16lo(wd[e]);
-        x[2 * e + 1] = bf16hi(wd[e]);
-      }
-      float ss = 0.f;
+      for (int j = 0; j < 4; ++j) x2[j] = f2pack(bf16lo(wd[j]), bf16hi(wd[j]));
+      uint64_t ss2 = mul2(x2[0], x2[0]);
 #pragma unroll
-      for (int e = 0; e < 8; ++e) ss = fmaf(x[e], x[e], ss);
+      for (int j = 1; j < 4; ++j) ss2 = fma2(x2[j], x2[j], ss2);
+      float s0, s1;
+      f2unpack(ss2, s0, s1);
+      float ss = s0 + s1;
       // the row's D/8 chunks sit in consecutive lanes: fold them (every lane
       // takes part, rows past L included, whose values are zero)
 #pragma unroll
       for (int off = 1; off < CH; off <<= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
       if (row < cnt) {
         const float inv = rsqrtf(ss * (1.0f / (float)D) + pro.eps);  // within 2 fp32 ulps
+        const uint64_t inv2 = f2pack(inv, inv);
         const int n = t0 + row;
         uint32_t o[4];
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
           const int pos = pax[j] == 0 ? pt : (pax[j] == 1 ? ph : pw);
           const float2 cs = __ldg(pro.table + pbase[j] + pos * pstride[j]);
-          const float xa = (x[2 * j] * inv) * wv[2 * j];
-          const float xb = (x[2 * j + 1] * inv) * wv[2 * j + 1];
-          const float y0 = fmaf(xa, cs.x, -xb * cs.y);
-          const float y1 = fmaf(xa, cs.y, xb * cs.x);
+          // u = x * w per channel; (y0, y1) = inv * (ua cos - ub sin, ua sin + ub cos)
+          float ua, ub;
+          f2unpack(mul2(x2[j], wp[j]), ua, ub);
+          const uint64_t p2 = mul2(f2pack(ub, ub), f2pack(-cs.y, cs.x));
+          const uint64_t y2 = mul2(fma2(f2pack(ua, ua), f2pack(cs.x, cs.y), p2), inv2);
+          float y0, y1;
+          f2unpack(y2, y0, y1);
           __nv_bfloat162 yb = __floats2bfloat162_rn(y0, y1);
           o[j] = *reinterpret_cast<uint32_t*>(&yb);
         }

@@ -101,16 +101,21 @@ __global__ void __launch_bounds__(256) ulysses_rows_kernel(UlyssesArgs a) {
 #pragma unroll
     for (int i = 0; i < kUlyPasses; ++i) {
       const uint32_t w[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
-      float m = 0.f;
+      // |x| maxima on bf16 pairs (exact), then over the row's lanes
+      __nv_bfloat162 m2 = __habs2(*reinterpret_cast<const __nv_bfloat162*>(&w[0]));
 #pragma unroll
-      for (int e = 0; e < 4; ++e) m = fmaxf(m, fmaxf(fabsf(bf16lo(w[e])), fabsf(bf16hi(w[e]))));
+      for (int e = 1; e < 4; ++e) m2 = __hmax2(m2, __habs2(*reinterpret_cast<const __nv_bfloat162*>(&w[e])));
+      float m = fmaxf(__low2float(m2), __high2float(m2));
 #pragma unroll
       for (int off = 1; off < CH; off <<= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
       const float inv = m > 0.f ? __fdiv_rn(448.0f, m) : 0.f;
-      const uint32_t c0 = e4m3x4(__fmul_rn(bf16lo(w[0]), inv), __fmul_rn(bf16hi(w[0]), inv),
-                                 __fmul_rn(bf16lo(w[1]), inv), __fmul_rn(bf16hi(w[1]), inv));
-      const uint32_t c1 = e4m3x4(__fmul_rn(bf16lo(w[2]), inv), __fmul_rn(bf16hi(w[2]), inv),
-                                 __fmul_rn(bf16lo(w[3]), inv), __fmul_rn(bf16hi(w[3]), inv));
+      // fl32(x * inv) in packed pairs (one rounding each, as __fmul_rn)
+      const uint64_t inv2 = f2pack(inv, inv);
+      float y[8];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) f2unpack(mul2(f2pack(bf16lo(w[e]), bf16hi(w[e])), inv2), y[2 * e], y[2 * e + 1]);
+      const uint32_t c0 = e4m3x4(y[0], y[1], y[2], y[3]);
+      const uint32_t c1 = e4m3x4(y[4], y[5], y[6], y[7]);
       if (live[i]) {
         *reinterpret_cast<uint2*>(a.codes + pr[i] * D + c * 8) = make_uint2(c0, c1);
         if (c == 0) a.scales[pr[i]] = m > 0.f ? __fdiv_rn(m, 448.0f) : 1.0f;
