@@ -36,15 +36,14 @@ def metric_for(workload, H, d, keep):
     return f"block-sparse attn ms & effective TFLOPS ({workload} grid, {H}\u00d7{d}, keep {keep:g})"
 
 
+# The attention kernel each mode launches and the sources it is built from.
+_CSRC = os.path.join(ROOT, "video_dit_dynamic_token_b200", "csrc")
+ATTN_KERNEL = {"int8fp8": ("sparse_attn_paired_kernel", ("attn.cuh", "attn_paired.cuh")),
+               "bf16": ("sparse_attn_kernel", ("attn.cuh",))}
 # DRAM bytes (read + write) of one full-size attention launch, from an ncu
-# capture, keyed by the SHA-256 of the kernel source it was taken on: when
-# attn.cuh changes the key no longer matches and the line reports null.
-ATTN_SRC = os.path.join(ROOT, "video_dit_dynamic_token_b200", "csrc", "attn.cuh")
-ATTN_DRAM_BYTES = {   # {sha256 of attn.cuh: (bytes per full 720p launch, how it was taken)}
-    "05b326c7b53ef8e933eb51083a6ff51c0abb28fbb8a2ea0d641653828126b804":
-        (5 * (236.935168e6 + 126.793984e6),
-         "ncu dram__bytes_read.sum + dram__bytes_write.sum of the 8-head 720p launch x 5 (traffic grows with the "
-         "heads)"),
+# capture, keyed by the SHA-256 of the kernel sources it was taken on: when
+# they change the key no longer matches and the line reports null.
+ATTN_DRAM_BYTES = {   # {sha256 of the mode's sources: (bytes per full 720p launch, how it was taken)}
 }
 
 # Dense MACs per clock per SM of one tcgen05 kind::i8 / kind::f8f6f4 M=128 MMA
@@ -53,10 +52,18 @@ TC_8BIT_MAC_PER_CLK_SM = 8192
 PEAKS_8BIT = os.path.join(ROOT, "MEASURED_PEAKS_8BIT.json")
 
 
-def attn_traffic():
+def attn_source_hash(mode):
     import hashlib
+    h = hashlib.sha256()
+    for f in ATTN_KERNEL[mode][1]:
+        with open(os.path.join(_CSRC, f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()
+
+
+def attn_traffic(mode="int8fp8"):
     try:
-        h = hashlib.sha256(open(ATTN_SRC, "rb").read()).hexdigest()
+        h = attn_source_hash(mode)
     except OSError:
         return None, "kernel source not found"
     if h in ATTN_DRAM_BYTES:
@@ -118,7 +125,7 @@ def attn_roofline(flops, ms, peaks, mode, d, sm_mhz=None, sms=148):
         peak, sustained = peaks["bf16"], peaks["bf16_sustained"]
         note = f"{peaks['source']} bf16 burst"
         mac = TC_8BIT_MAC_PER_CLK_SM // 2
-    out = {"bound": "tensor", "kernel": f"sparse_attn_kernel<{d},{mode}>", "achieved": round(achieved, 1),
+    out = {"bound": "tensor", "kernel": f"{ATTN_KERNEL[mode][0]}<{d},{mode}>", "achieved": round(achieved, 1),
            "peak": round(peak, 1), "unit": "TFLOP/s", "frac": round(achieved / peak, 3), "peak_note": note,
            "frac_of_sustained": round(achieved / sustained, 3), "sustained_peak": round(sustained, 1)}
     if sm_mhz:
@@ -437,8 +444,8 @@ def run_ours(args, rank, world, local_rank):
     esz = 1 if mode == "int8fp8" else 2
     attn_bytes = 3 * B * H * L * d * esz + B * H * L * d * 2 + B * H * nB * k * 4
     roof = attn_roofline(flops, attn_ms, peaks, mode, d, (clocks or {}).get("sm_mhz"))
-    traffic, traffic_note = attn_traffic()
-    if args.heads or mode != MODE or args.workload != WORKLOAD or args.keep:
+    traffic, traffic_note = attn_traffic(mode)
+    if args.heads or args.workload != WORKLOAD or args.keep:
         traffic, traffic_note = None, "captured for the 720p headline launch only"
     roof.update({"traffic": traffic, "traffic_note": traffic_note, "algorithmic_bytes": int(attn_bytes)})
     out = {
@@ -515,11 +522,9 @@ def run_ulysses_share(args):
     g = torch.Generator(device=dev).manual_seed(0)
     q, k, v = ((torch.randn(B, Lr, H, d, generator=g, device=dev)).to(torch.bfloat16) for _ in range(3))
     qv, kv, vv = (x.permute(0, 2, 1, 3) for x in (q, k, v))
-    c = torch.empty((N, B, Hr, Lr, 3, d), dtype=torch.uint8, device=dev)
-    sc = torch.empty((N, B, Hr, Lr, 3), dtype=torch.float32, device=dev)
+    pay = ulysses.new_payload(N, B, Hr, Lr, d, 3, dev)
     qh, kh, vh = (torch.empty((B, Hr, L, d), dtype=torch.bfloat16, device=dev) for _ in range(3))
-    oc = torch.empty((N, B, Hr, Lr, d), dtype=torch.uint8, device=dev)
-    osc = torch.empty((N, B, Hr, Lr), dtype=torch.float32, device=dev)
+    pay_o = ulysses.new_payload(N, B, Hr, Lr, d, 1, dev)
     out = torch.empty_like(q)
     ws = torch.empty(lx.lx_sparse_attn_ws_size(qh, keep, args.mode), dtype=torch.uint8, device=dev)
     oh = torch.empty_like(qh)
@@ -530,15 +535,15 @@ def run_ulysses_share(args):
             if ev is not None:
                 ev[i].record()
         mark(0)
-        ulysses.pack_qkv(qv, kv, vv, N, 0, Hr, c, sc)
+        ulysses.pack_qkv(qv, kv, vv, N, 0, Hr, pay)
         mark(1)
-        ulysses.unpack_qkv(c, sc, N, qh, kh, vh)
+        ulysses.unpack_qkv(pay, N, qh, kh, vh)
         mark(2)
         lx.lx_sparse_attn(qh, kh, vh, keep, args.mode, out=oh, ws=ws)
         mark(3)
-        ulysses.pack_o(oh, N, oc, osc)
+        ulysses.pack_o(oh, N, pay_o)
         mark(4)
-        ulysses.unpack_o(oc, osc, N, 0, Hr, out.permute(0, 2, 1, 3))
+        ulysses.unpack_o(pay_o, N, 0, Hr, out.permute(0, 2, 1, 3))
         mark(5)
 
     for _ in range(args.warmup):

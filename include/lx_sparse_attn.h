@@ -191,29 +191,39 @@ lx_status lx_pool_quantize_qk_smooth(const lx_bhld* Q, const lx_bhld* K, const f
  * (Hr = H / N) of all L = N Lr tokens after it.  One FP8 scale per (token,
  * head, tensor) row of D values: s = absmax/448 (1 for an all-zero row), code
  * = E4M3_rn_satfinite(fl32(x * fl32(448/absmax))); the receiver writes
- * bf16(fl32(decode(code) * s)).  The collective itself is the caller's (one
- * all-to-all with equal splits over the leading N of each buffer); these calls
- * build and read its buffers.
+ * bf16(fl32(decode(code) * s)).  The collective itself is the caller's: one
+ * all-to-all with equal splits over a payload of N segments; these calls
+ * build and read the payload.
  *
+ * Payload: N segments of seg bytes (lx_ulysses_segment_bytes), segment n for
+ * (pack) or from (unpack) rank n.  A segment holds the codes, uint8
+ * [B][hc][Lr][X][D] (X = 3 tensors q, k, v for the Q/K/V payload, X = 1 for
+ * the output payload), then, from byte offset roundup16(B hc Lr X D), the
+ * scales, fp32 [B][hc][Lr][X]; seg = that offset + roundup16(4 B hc Lr X).
+ *
+ * lx_ulysses_segment_bytes: seg for the given sizes (tensors = X = 3 or 1);
+ * LX_ERR_INVALID for sizes below 1, D other than 64 or 128, or another X.
  * lx_ulysses_pack_qkv: q, k, v this rank's shard viewed as [B, H, Lr, D] (any
- * strides, e.g. the [B, Lr, H, D] layout); sends heads h0 .. h0+hc-1 of each
- * destination's range: codes [N][B][hc][Lr][3][D] uint8, scales
- * [N][B][hc][Lr][3] fp32.
- * lx_ulysses_unpack_qkv: the received buffers (same layout, slice n from rank
- * n) into q, k, v [B, hc, L, D] (L divisible by N; token n Lr + t from rank n).
- * lx_ulysses_pack_o: the attention output o [B, hc, L, D] of those heads:
- * codes [N][B][hc][Lr][D], scales [N][B][hc][Lr], slice n holding rank n's
- * tokens.
- * lx_ulysses_unpack_o: the received output buffers into this rank's shard
+ * strides, e.g. the [B, Lr, H, D] layout); segment n carries heads
+ * n Hr + h0 .. n Hr + h0 + hc - 1 of the shard.
+ * lx_ulysses_unpack_qkv: the received Q/K/V payload (segment n from rank n,
+ * hc = q's head count, Lr = L / N) into q, k, v [B, hc, L, D] (token n Lr + t
+ * from rank n).
+ * lx_ulysses_pack_o: the attention output o [B, hc, L, D] of those heads;
+ * segment n holds rank n's tokens (Lr = L / N).
+ * lx_ulysses_unpack_o: the received output payload into this rank's shard
  * out [B, H, Lr, D] (any strides), heads n Hr + h0 .. n Hr + h0 + hc - 1 from
- * rank n.  Pointers 16-byte aligned; errors as elsewhere. */
+ * segment n.  The payload pointer 16-byte aligned (LX_ERR_ALIGN otherwise);
+ * shapes as stated (LX_ERR_INVALID otherwise); the payload is the caller's
+ * device memory, N seg bytes. */
+lx_status lx_ulysses_segment_bytes(int64_t B, int64_t hc, int64_t Lr, int64_t D, int64_t tensors, size_t* seg_bytes);
 lx_status lx_ulysses_pack_qkv(const lx_bhld* q, const lx_bhld* k, const lx_bhld* v, int64_t N, int64_t h0, int64_t hc,
-                              uint8_t* codes, float* scales, cudaStream_t stream);
-lx_status lx_ulysses_unpack_qkv(const uint8_t* codes, const float* scales, int64_t N, const lx_bhld* q,
-                                const lx_bhld* k, const lx_bhld* v, cudaStream_t stream);
-lx_status lx_ulysses_pack_o(const lx_bhld* o, int64_t N, uint8_t* codes, float* scales, cudaStream_t stream);
-lx_status lx_ulysses_unpack_o(const uint8_t* codes, const float* scales, int64_t N, int64_t h0, int64_t hc,
-                              const lx_bhld* out, cudaStream_t stream);
+                              uint8_t* payload, cudaStream_t stream);
+lx_status lx_ulysses_unpack_qkv(const uint8_t* payload, int64_t N, const lx_bhld* q, const lx_bhld* k,
+                                const lx_bhld* v, cudaStream_t stream);
+lx_status lx_ulysses_pack_o(const lx_bhld* o, int64_t N, uint8_t* payload, cudaStream_t stream);
+lx_status lx_ulysses_unpack_o(const uint8_t* payload, int64_t N, int64_t h0, int64_t hc, const lx_bhld* out,
+                              cudaStream_t stream);
 
 /* Step a3 -- FP8 E4M3 V ("600倍加速…", §高效推理算子: "V FP8").
  * vc: uint8 [B,H,L,D] contiguous E4M3 codes; vs: fp32 [B,H,D] scales =

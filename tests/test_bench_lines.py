@@ -18,6 +18,7 @@ def test_attn_roofline_int8_and_bf16():
     assert "tcgen05_peak_at_clock" not in r
     b = bench.attn_roofline(2.0e12, 2.0, PEAKS, "bf16", 128)
     assert b["peak"] == 1628.7 and b["kernel"] == "sparse_attn_kernel<128,bf16>"
+    assert r["kernel"] == "sparse_attn_paired_kernel<128,int8fp8>"
     assert b["frac_of_sustained"] == round(1000.0 / 1380.3, 3)
 
 
@@ -39,11 +40,19 @@ def test_peaks_without_8bit_file_fall_back_to_twice_bf16_burst(tmp_path, monkeyp
 
 def test_attn_traffic_is_keyed_by_kernel_source(monkeypatch):
     import hashlib
-    h = hashlib.sha256(open(bench.ATTN_SRC, "rb").read()).hexdigest()
-    monkeypatch.setattr(bench, "ATTN_DRAM_BYTES", {"0" * 64: (1, "stale")})
-    assert bench.attn_traffic()[0] is None
-    monkeypatch.setattr(bench, "ATTN_DRAM_BYTES", {h: (123, "capture")})
-    assert bench.attn_traffic() == (123, "capture")
+    import os
+    for mode in ("int8fp8", "bf16"):
+        h = hashlib.sha256()
+        for f in bench.ATTN_KERNEL[mode][1]:
+            h.update(open(os.path.join(bench._CSRC, f), "rb").read())
+        h = h.hexdigest()
+        assert bench.attn_source_hash(mode) == h
+        monkeypatch.setattr(bench, "ATTN_DRAM_BYTES", {"0" * 64: (1, "stale")})
+        assert bench.attn_traffic(mode)[0] is None
+        monkeypatch.setattr(bench, "ATTN_DRAM_BYTES", {h: (123, "capture")})
+        assert bench.attn_traffic(mode) == (123, "capture")
+    # the two modes run different kernels, so their keys differ
+    assert bench.attn_source_hash("int8fp8") != bench.attn_source_hash("bf16")
 
 
 def test_ulysses_cpu_sample_combines_exchange_and_attention():

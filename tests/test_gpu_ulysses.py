@@ -1,6 +1,7 @@
 """Light-Ulysses exchange kernels against the oracle, bit for bit: N virtual
-ranks on one GPU, the all-to-all emulated by slicing; and the whole
-ulysses_sparse_attn on a one-rank NCCL group."""
+ranks on one GPU, the all-to-all emulated by gathering segment r of every
+rank's payload for rank r; and the whole ulysses_sparse_attn on a one-rank
+NCCL group."""
 import datetime
 import socket
 
@@ -33,29 +34,29 @@ def test_qkv_and_output_exchange_bit_exact(N, B, Lr, H, D):
         sends = []
         for r in range(N):
             qv, kv, vv = (x.permute(0, 2, 1, 3) for x in shards[r])
-            c = torch.empty((N, B, hc, Lr, 3, D), dtype=torch.uint8, device=DEV)
-            s = torch.empty((N, B, hc, Lr, 3), dtype=torch.float32, device=DEV)
-            ulysses.pack_qkv(qv, kv, vv, N, h0, hc, c, s)
-            sends.append((c, s))
+            pay = ulysses.new_payload(N, B, hc, Lr, D, 3, DEV)
+            ulysses.pack_qkv(qv, kv, vv, N, h0, hc, pay)
+            sends.append(pay)
+            c, s = ulysses.payload_views(pay, B, hc, Lr, D, 3)
             heads = [n * Hr + h0 + j for n in range(N) for j in range(hc)]
             rc, rs = oracle.pack_qkv_ref(*(x[:, :, heads].cpu() for x in shards[r]), N)
             assert np.array_equal(to_np(c), rc) and np.array_equal(to_np(s), rs)
         for r in range(N):
-            rc = torch.stack([sends[n][0][r] for n in range(N)])
-            rs = torch.stack([sends[n][1][r] for n in range(N)])
+            recv = torch.stack([sends[n][r] for n in range(N)])
+            rc, rs = ulysses.payload_views(recv, B, hc, Lr, D, 3)
             qh, kh, vh = (torch.empty((B, hc, N * Lr, D), dtype=torch.bfloat16, device=DEV) for _ in range(3))
-            ulysses.unpack_qkv(rc, rs, N, qh, kh, vh)
+            ulysses.unpack_qkv(recv, N, qh, kh, vh)
             want = oracle.unpack_qkv_ref(to_np(rc), to_np(rs))
             for got, w in zip((qh, kh, vh), want):
                 assert np.array_equal(to_np(got.float()).astype(np.float64), w)
             # the way back, with the received V standing in for the output
-            oc = torch.empty((N, B, hc, Lr, D), dtype=torch.uint8, device=DEV)
-            os_ = torch.empty((N, B, hc, Lr), dtype=torch.float32, device=DEV)
-            ulysses.pack_o(vh, N, oc, os_)
+            pay_o = ulysses.new_payload(N, B, hc, Lr, D, 1, DEV)
+            ulysses.pack_o(vh, N, pay_o)
+            oc, os_ = ulysses.payload_views(pay_o, B, hc, Lr, D, 1)
             c2, s2 = oracle.pack_o_ref(vh.cpu(), N)
             assert np.array_equal(to_np(oc), c2) and np.array_equal(to_np(os_), s2)
             out = torch.zeros((B, Lr, H, D), dtype=torch.bfloat16, device=DEV)
-            ulysses.unpack_o(oc, os_, N, h0, hc, out.permute(0, 2, 1, 3))
+            ulysses.unpack_o(pay_o, N, h0, hc, out.permute(0, 2, 1, 3))
             y = oracle.unpack_o_ref(c2, s2)                       # [B, Lr, N*hc, D]
             for n in range(N):
                 for j in range(hc):
@@ -80,16 +81,14 @@ def test_ulysses_sparse_attn_one_rank_nccl():
     assert lx.lx_last_device_status() == 0
     # the same steps called one by one (one chunk of all heads: the attention is per head)
     qv, kv, vv = (x.permute(0, 2, 1, 3) for x in (q, k, v))
-    c = torch.empty((1, B, H, L, 3, D), dtype=torch.uint8, device=DEV)
-    s = torch.empty((1, B, H, L, 3), dtype=torch.float32, device=DEV)
-    ulysses.pack_qkv(qv, kv, vv, 1, 0, H, c, s)
+    pay = ulysses.new_payload(1, B, H, L, D, 3, DEV)
+    ulysses.pack_qkv(qv, kv, vv, 1, 0, H, pay)
     qh, kh, vh = (torch.empty((B, H, L, D), dtype=torch.bfloat16, device=DEV) for _ in range(3))
-    ulysses.unpack_qkv(c, s, 1, qh, kh, vh)
+    ulysses.unpack_qkv(pay, 1, qh, kh, vh)
     oh, _ = lx.lx_sparse_attn(qh, kh, vh, keep, "int8fp8")
-    oc = torch.empty((1, B, H, L, D), dtype=torch.uint8, device=DEV)
-    os_ = torch.empty((1, B, H, L), dtype=torch.float32, device=DEV)
-    ulysses.pack_o(oh, 1, oc, os_)
+    pay_o = ulysses.new_payload(1, B, H, L, D, 1, DEV)
+    ulysses.pack_o(oh, 1, pay_o)
     want = torch.empty_like(q)
-    ulysses.unpack_o(oc, os_, 1, 0, H, want.permute(0, 2, 1, 3))
+    ulysses.unpack_o(pay_o, 1, 0, H, want.permute(0, 2, 1, 3))
     torch.cuda.synchronize()
     assert torch.equal(out, want)

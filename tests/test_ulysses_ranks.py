@@ -29,27 +29,35 @@ def _shards(world, B, Lr, H, D):
 
 def _oracle_ops():
     import oracle
-    from video_dit_dynamic_token_b200.ulysses import UlyssesOps
+    from video_dit_dynamic_token_b200.ulysses import UlyssesOps, payload_views
 
-    def pack_qkv(qv, kv, vv, N, h0, hc, codes, scales):
+    def pack_qkv(qv, kv, vv, N, h0, hc, payload):
         # heads h0 .. h0+hc-1 of each destination's range, in destination order
-        Hr = qv.shape[1] // N
+        B, H, Lr, D = qv.shape
+        Hr = H // N
         heads = [n * Hr + h0 + j for n in range(N) for j in range(hc)]
         sub = [x[:, heads].permute(0, 2, 1, 3).float().numpy() for x in (qv, kv, vv)]   # [B, Lr, N*hc, D]
         c, s = oracle.pack_qkv_ref(sub[0], sub[1], sub[2], N)
+        codes, scales = payload_views(payload, B, hc, Lr, D, 3)
         codes.copy_(torch.from_numpy(c))
         scales.copy_(torch.from_numpy(s))
 
-    def unpack_qkv(codes, scales, N, qh, kh, vh):
+    def unpack_qkv(payload, N, qh, kh, vh):
+        B, hc, L, D = qh.shape
+        codes, scales = payload_views(payload, B, hc, L // N, D, 3)
         for dst, y in zip((qh, kh, vh), oracle.unpack_qkv_ref(codes.numpy(), scales.numpy())):
             dst.copy_(torch.from_numpy(y).to(torch.bfloat16))
 
-    def pack_o(oh, N, codes, scales):
+    def pack_o(oh, N, payload):
+        B, hc, L, D = oh.shape
         c, s = oracle.pack_o_ref(oh.float().numpy(), N)
+        codes, scales = payload_views(payload, B, hc, L // N, D, 1)
         codes.copy_(torch.from_numpy(c))
         scales.copy_(torch.from_numpy(s))
 
-    def unpack_o(codes, scales, N, h0, hc, outv):
+    def unpack_o(payload, N, h0, hc, outv):
+        B, H, Lr, D = outv.shape
+        codes, scales = payload_views(payload, B, hc, Lr, D, 1)
         y = oracle.unpack_o_ref(codes.numpy(), scales.numpy())      # [B, Lr, N*hc, D]
         Hr = outv.shape[1] // N
         for n in range(N):
@@ -110,3 +118,28 @@ def test_head_chunks_cover_all_heads():
             ch = head_chunks(Hr, n)
             assert sum(hc for _, hc in ch) == Hr and ch[0][0] == 0
             assert all(ch[i][0] + ch[i][1] == ch[i + 1][0] for i in range(len(ch) - 1))
+
+
+def test_payload_layout_matches_the_library():
+    """The host-side segment layout equals lx_ulysses_segment_bytes (a host
+    call), and the code and scale views tile each segment without overlap."""
+    sys.path.insert(0, ROOT)
+    import ctypes
+    from video_dit_dynamic_token_b200 import _abi
+    from video_dit_dynamic_token_b200.ulysses import payload_views, segment_layout
+    lib = _abi.load()
+    for B, hc, Lr, D, X in [(1, 2, 96, 128, 3), (2, 3, 41, 64, 3), (1, 1, 7, 64, 1), (2, 5, 1, 128, 1)]:
+        seg = ctypes.c_size_t(0)
+        assert lib.lx_ulysses_segment_bytes(B, hc, Lr, D, X, ctypes.byref(seg)) == 0
+        rows, sc_off, nbytes = segment_layout(B, hc, Lr, D, X)
+        assert seg.value == nbytes and sc_off % 16 == 0 and nbytes % 16 == 0
+        assert rows * D <= sc_off < sc_off + 4 * rows <= nbytes
+        pay = torch.zeros((3, nbytes), dtype=torch.uint8)
+        c, s = payload_views(pay, B, hc, Lr, D, X)
+        c.fill_(1)
+        s.view(torch.int32).fill_(0x01010101)   # no zero byte in any scale
+        used = (pay != 0).sum(dim=1)
+        assert used.tolist() == [rows * D + 4 * rows] * 3
+    bad = ctypes.c_size_t(0)
+    assert lib.lx_ulysses_segment_bytes(1, 1, 1, 96, 3, ctypes.byref(bad)) != 0
+    assert lib.lx_ulysses_segment_bytes(1, 1, 1, 128, 2, ctypes.byref(bad)) != 0

@@ -63,10 +63,11 @@ SIGNATURES = {
     "lx_sparse_attn_fwd": [_P(LxBhld), _P(LxBhld), _P(LxBhld), _P(LxPlan), ctypes.c_int, _P(LxBhld), _vp, _c_sz, _vp],
     "lx_sparse_attn_ws_size": [_P(LxBhld), _dbl, ctypes.c_int, _P(_c_sz)],
     "lx_sparse_attn": [_P(LxBhld), _P(LxBhld), _P(LxBhld), _dbl, ctypes.c_int, _P(LxPlan), _P(LxBhld), _vp, _c_sz, _vp],
-    "lx_ulysses_pack_qkv": [_P(LxBhld), _P(LxBhld), _P(LxBhld), _c_i64, _c_i64, _c_i64, _vp, _vp, _vp],
-    "lx_ulysses_unpack_qkv": [_vp, _vp, _c_i64, _P(LxBhld), _P(LxBhld), _P(LxBhld), _vp],
-    "lx_ulysses_pack_o": [_P(LxBhld), _c_i64, _vp, _vp, _vp],
-    "lx_ulysses_unpack_o": [_vp, _vp, _c_i64, _c_i64, _c_i64, _P(LxBhld), _vp],
+    "lx_ulysses_segment_bytes": [_c_i64, _c_i64, _c_i64, _c_i64, _c_i64, _P(_c_sz)],
+    "lx_ulysses_pack_qkv": [_P(LxBhld), _P(LxBhld), _P(LxBhld), _c_i64, _c_i64, _c_i64, _vp, _vp],
+    "lx_ulysses_unpack_qkv": [_vp, _c_i64, _P(LxBhld), _P(LxBhld), _P(LxBhld), _vp],
+    "lx_ulysses_pack_o": [_P(LxBhld), _c_i64, _vp, _vp],
+    "lx_ulysses_unpack_o": [_vp, _c_i64, _c_i64, _c_i64, _P(LxBhld), _vp],
     "lx_nvfp4_sizes": [_c_i64, _c_i64, _P(_c_sz), _P(_c_sz)],
     "lx_nvfp4_quantize": [_vp, _c_i64, _c_i64, _c_i64, ctypes.c_int, _vp, _vp, _vp, _vp],
     "lx_nvfp4_gemm": [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _c_i64, _c_i64, _c_i64, _vp, _c_i64, _vp],

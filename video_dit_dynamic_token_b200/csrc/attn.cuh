@@ -5,6 +5,11 @@
 // inside; §高效推理算子: Q/K INT8 and V FP8.  "Run Wan2.2-A14B on One RTX 5090:
 // 720p Video in 3.8s", §3 Dynamic sparse attention: the same in English.
 //
+// Per-step form: the kernel that BF16 calls run.  INT8/FP8 calls run the
+// paired-S form of attn_paired.cuh, measured 2-4 % faster in that mode.  This
+// kernel's INT8/FP8 form is complete (it passed the INT8/FP8 parity tests
+// when the two were compared) but the library does not launch it.
+//
 // Tile: one CTA owns two adjacent 64-row query blocks (2p, 2p+1), run as two
 // independent M=64 streams A and B in lockstep; two CTAs share an SM.  Step c
 // computes query block 2p against its c-th kept key block and query block
@@ -18,10 +23,11 @@
 //
 // Pipeline (per step c, every buffer two-deep by step parity): K and V blocks
 // of both streams in two-stage rings, S(c) (M=64, N=64) in TMEM columns
-// [64 (c & 1), +64), P(c) in shared memory.  S(c+2) is issued as soon as the
-// softmax has read S(c), early in step c, and its K blocks load while S(c)
-// computes; P.V(c) is issued when P(c) is written.  The softmax waits for
-// P.V(c-1) only when one of its warp's rows must rescale O.
+// [64 (c & 1), +64), P(c) in shared memory.  S(c+2) is issued once the
+// softmax has read S(c) (BF16: right after the load; INT8: after the
+// exponentials, under which the restart of its columns completes), and its K
+// blocks load while S(c) computes; P.V(c) is issued when P(c) is written.  The
+// softmax waits for P.V(c-1) only when one of its warp's rows must rescale O.
 //
 // Roles (6 warps): warp 0 = TMA producer (Q once, then K and V blocks);
 // warp 1 = TMEM allocator + MMA issuer (S_A, S_B = Q K^T into the S columns,
@@ -73,6 +79,7 @@ struct AttnCfg {
   static constexpr uint32_t IDESC_PV =
       instr_desc(IDESC_DF32, I8 ? IDESC_E4M3 : IDESC_BF16, I8 ? IDESC_E4M3 : IDESC_BF16, 0, 1, 64, D);
   static constexpr int KEYS_PER_MMA = 32 / ESZ;           // 32 bytes of K per instruction
+  static constexpr int THREADS = 192;                     // producer, MMA, four softmax warps
 };
 
 struct AttnParams {
@@ -107,7 +114,7 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, const 
 }
 
 template <int D, bool I8>
-__global__ void __launch_bounds__(192, I8 ? 2 : 1)
+__global__ void __launch_bounds__(AttnCfg<D, I8>::THREADS, I8 ? 2 : 1)
     sparse_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                        const __grid_constant__ CUtensorMap tmV, const AttnParams prm) {
   using C = AttnCfg<D, I8>;
@@ -339,9 +346,15 @@ __global__ void __launch_bounds__(192, I8 ? 2 : 1)
     mbar_arrive(&bar_sfree[0]);
     mbar_arrive(&bar_sfree[1]);
     bool ok = true;
+    int j_next = n > 0 ? my_idx[0] : 0;
+    float sk_next = (I8 && n > 0) ? my_skl[0] : 1.f;
     for (int c = 0; c < n; ++c) {
-      const int j = my_idx[c];
-      const float skj = I8 ? my_skl[c] : 1.f;
+      const int j = j_next;
+      const float skj = sk_next;
+      if (c + 1 < n) {
+        j_next = my_idx[c + 1];
+        if constexpr (I8) sk_next = my_skl[c + 1];
+      }
       const int half = c & 1;  // S buffer and P tiles of this step
       const uint32_t s_addr = lane_addr + C::S_COL + 64 * half;
       ok = warp_wait(&bar_sfull[half], (c >> 1) & 1, &abort_flag, prm.limit_ns);
@@ -355,18 +368,19 @@ __global__ void __launch_bounds__(192, I8 ? 2 : 1)
         tmem_ld32(s_addr + 32, hi);
         tmem_wait_ld();
       }
-      // INT8: restart these columns at the magic value, then hand the S
-      // buffer back to the MMA warp: S(c+2) runs while this step's softmax runs
+      // INT8: restart these columns at the magic value; the store completes
+      // under the block max and the exponentials, and the S buffer goes back to
+      // the MMA warp after them (S(c+2) is not needed for two steps)
       if constexpr (I8) {
         uint32_t mg[32];
 #pragma unroll
         for (int i = 0; i < 32; ++i) mg[i] = kMagicBits;
         tmem_st32(s_addr, mg);
         tmem_st32(s_addr + 32, mg);
-        tmem_wait_st();
+      } else {
+        tc_fence_before();
+        mbar_arrive(&bar_sfree[half]);
       }
-      tc_fence_before();
-      mbar_arrive(&bar_sfree[half]);
       const int nvalid = (j == prm.nB - 1) ? (prm.L - j * kBlock) : kBlock;
       float sc = prm.scale_log2;
       if constexpr (I8) sc *= sq * skj;
@@ -440,6 +454,11 @@ __global__ void __launch_bounds__(192, I8 ? 2 : 1)
 #pragma unroll
         for (int i = 0; i < PW; ++i) pk[i] = 0u;
       }
+      if constexpr (I8) {
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(&bar_sfree[half]);
+      }
       // P tiles of parity c & 1 are free once P.V(c-2) is complete
       if (c >= 2) {
         ok = warp_wait(&bar_odone[half], ((c - 2) >> 1) & 1, &abort_flag, prm.limit_ns);
@@ -455,19 +474,29 @@ __global__ void __launch_bounds__(192, I8 ? 2 : 1)
           tc_fence_after();
           const float f = need_rescale ? alpha : 1.f;
           const uint64_t f2 = f2pack(f, f);
+          // BF16 (one CTA per SM, registers to spare): two 32-column loads in
+          // flight per round trip; INT8 (two CTAs per SM): one
+          constexpr int RW = I8 ? 1 : 2;
 #pragma unroll
-          for (int cc = 0; cc < D; cc += 32) {
-            uint32_t o[32];
-            tmem_ld32(lane_addr + C::O_COL + cc, o);
+          for (int cc = 0; cc < D; cc += 32 * RW) {
+            uint32_t o[RW][32];
+#pragma unroll
+            for (int hh = 0; hh < RW; ++hh)
+              if (cc + 32 * hh < D) tmem_ld32(lane_addr + C::O_COL + cc + 32 * hh, o[hh]);
             tmem_wait_ld();
 #pragma unroll
-            for (int i = 0; i < 32; i += 2) {
-              float a, b;
-              f2unpack(mul2(f2pack(__uint_as_float(o[i]), __uint_as_float(o[i + 1])), f2), a, b);
-              o[i] = __float_as_uint(a);
-              o[i + 1] = __float_as_uint(b);
+            for (int hh = 0; hh < RW; ++hh) {
+              if (cc + 32 * hh < D) {
+#pragma unroll
+                for (int i = 0; i < 32; i += 2) {
+                  float a, b;
+                  f2unpack(mul2(f2pack(__uint_as_float(o[hh][i]), __uint_as_float(o[hh][i + 1])), f2), a, b);
+                  o[hh][i] = __float_as_uint(a);
+                  o[hh][i + 1] = __float_as_uint(b);
+                }
+                tmem_st32(lane_addr + C::O_COL + cc + 32 * hh, o[hh]);
+              }
             }
-            tmem_st32(lane_addr + C::O_COL + cc, o);
           }
           tmem_wait_st();
         }

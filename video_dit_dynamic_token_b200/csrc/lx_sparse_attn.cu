@@ -14,6 +14,7 @@
 #include "ulysses.cuh"
 #include "nvfp4.cuh"
 #include "attn.cuh"
+#include "attn_paired.cuh"
 
 namespace {
 
@@ -203,6 +204,40 @@ lx_status launch_quant_v(const lx_bhld* V, uint8_t* vc, float* vs, uint32_t* ama
   return launch_status();
 }
 
+// INT8/FP8 attention: the paired-S kernel (attn_paired.cuh)
+template <int D>
+lx_status launch_attn_paired(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const lx_plan* plan,
+                             const lx_bhld* O, const float* qs, const float* ks, const float* vs, cudaStream_t s) {
+  using C = lx::AttnPairCfg<D, true>;
+  const int64_t nB = plan->nB;
+  // the two kept lists follow the tiles
+  const size_t smem = 1024 + C::OFF_IDX + 2 * sizeof(int32_t) * (size_t)plan->k;
+  if (smem > 227 * 1024) return LX_ERR_UNSUPPORTED;
+  if (cudaFuncSetAttribute(lx::sparse_attn_paired_kernel<D, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)smem) != cudaSuccess)
+    return LX_ERR_CUDA;
+  lx::AttnParams p;
+  p.idx = plan->idx;
+  p.k = (int)plan->k;
+  p.nB = (int)nB;
+  p.L = (int)plan->L;
+  p.H = (int)plan->H;
+  p.o = reinterpret_cast<__nv_bfloat16*>(O->data);
+  p.osB = O->sB;
+  p.osH = O->sH;
+  p.osL = O->sL;
+  p.sq = qs;
+  p.sk = ks;
+  p.sv = vs;
+  p.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)D));
+  p.limit_ns = kWaitLimitNs;
+  // one CTA per (pair of query blocks, b*h), head-major so that a head's K/V stays in L2
+  dim3 grid((unsigned)((nB + 1) / 2), (unsigned)(plan->B * plan->H));
+  lx::sparse_attn_paired_kernel<D, true><<<grid, 192, smem, s>>>(mq, mk, mv, p);
+  return launch_status();
+}
+
+// BF16 attention: the per-step kernel (attn.cuh)
 template <int D, bool I8>
 lx_status launch_attn(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const lx_plan* plan,
                       const lx_bhld* O, const float* qs, const float* ks, const float* vs, cudaStream_t s) {
@@ -231,7 +266,7 @@ lx_status launch_attn(const CUtensorMap& mq, const CUtensorMap& mk, const CUtens
   p.limit_ns = kWaitLimitNs;
   // one CTA per (pair of query blocks, b*h), head-major so that a head's K/V stays in L2
   dim3 grid((unsigned)((nB + 1) / 2), (unsigned)(plan->B * plan->H));
-  lx::sparse_attn_kernel<D, I8><<<grid, 192, smem, s>>>(mq, mk, mv, p);
+  lx::sparse_attn_kernel<D, I8><<<grid, C::THREADS, smem, s>>>(mq, mk, mv, p);
   return launch_status();
 }
 
@@ -258,7 +293,7 @@ lx_status attn_i8_impl(const int8_t* qc, const float* qs, const int8_t* kc, cons
       !make_map(&mk, kc, dt, 1, B, H, L, D, sB, sH, sL, D, 64) ||
       !make_map(&mv, vc, dt, 1, B, H, L, D, sB, sH, sL, D, 64))
     return LX_ERR_CUDA;
-  return launch_attn<D, true>(mq, mk, mv, plan, O, qs, ks, vs, s);
+  return launch_attn_paired<D>(mq, mk, mv, plan, O, qs, ks, vs, s);
 }
 
 struct FwdWs {
@@ -750,87 +785,109 @@ lx_status lx_debug_wait_timeout(uint64_t limit_ns, cudaStream_t stream) {
 }
 
 // ---------------------------------------------------------------- Light-Ulysses exchange
+namespace {
+// rows of one destination's segment, its scale offset and its size (16-byte rounded)
+void ulysses_segment(int64_t B, int64_t hc, int64_t Lr, int64_t D, int64_t X, long long* rows_r, long long* sc_off,
+                     long long* seg) {
+  *rows_r = (long long)B * hc * Lr * X;
+  *sc_off = (*rows_r * D + 15) / 16 * 16;
+  *seg = *sc_off + (*rows_r * 4 + 15) / 16 * 16;
+}
+}  // namespace
+
+lx_status lx_ulysses_segment_bytes(int64_t B, int64_t hc, int64_t Lr, int64_t D, int64_t tensors, size_t* seg_bytes) {
+  if (!seg_bytes || B < 1 || hc < 1 || Lr < 1 || (D != 64 && D != 128) || (tensors != 1 && tensors != 3))
+    return LX_ERR_INVALID;
+  long long rows_r, sc_off, seg;
+  ulysses_segment(B, hc, Lr, D, tensors, &rows_r, &sc_off, &seg);
+  *seg_bytes = (size_t)seg;
+  return LX_OK;
+}
+
 lx_status lx_ulysses_pack_qkv(const lx_bhld* q, const lx_bhld* k, const lx_bhld* v, int64_t N, int64_t h0, int64_t hc,
-                              uint8_t* codes, float* scales, cudaStream_t stream) {
+                              uint8_t* payload, cudaStream_t stream) {
   lx_status st;
   if ((st = check_bhld(q)) != LX_OK || (st = check_bhld(k)) != LX_OK || (st = check_bhld(v)) != LX_OK) return st;
-  if (!same_shape(q, k) || !same_shape(q, v) || !codes || !scales) return LX_ERR_INVALID;
+  if (!same_shape(q, k) || !same_shape(q, v) || !payload) return LX_ERR_INVALID;
   if (N < 1 || q->H % N != 0 || h0 < 0 || hc < 1 || h0 + hc > q->H / N) return LX_ERR_INVALID;
-  if (!al16(codes) || !al16(scales)) return LX_ERR_ALIGN;
+  if (!al16(payload)) return LX_ERR_ALIGN;
   lx::UlyssesArgs a{};
   a.x[0] = rw(q);
   a.x[1] = rw(k);
   a.x[2] = rw(v);
-  a.codes = codes;
-  a.scales = scales;
+  a.payload = payload;
+  long long rows_r;
+  ulysses_segment(q->B, hc, q->L, q->D, 3, &rows_r, &a.sc_off, &a.seg);
   a.N = (int)N;
   a.B = (int)q->B;
   a.Hr = (int)(q->H / N);
   a.Hc = (int)hc;
   a.h0 = (int)h0;
   a.Lr = (int)q->L;
-  a.rows = (long long)N * q->B * hc * q->L * 3;
+  a.rows = (long long)N * rows_r;
   return launch_ulysses<lx::kPackQKV>(a, q->D, stream);
 }
 
-lx_status lx_ulysses_unpack_qkv(const uint8_t* codes, const float* scales, int64_t N, const lx_bhld* q,
-                                const lx_bhld* k, const lx_bhld* v, cudaStream_t stream) {
+lx_status lx_ulysses_unpack_qkv(const uint8_t* payload, int64_t N, const lx_bhld* q, const lx_bhld* k,
+                                const lx_bhld* v, cudaStream_t stream) {
   lx_status st;
   if ((st = check_bhld(q)) != LX_OK || (st = check_bhld(k)) != LX_OK || (st = check_bhld(v)) != LX_OK) return st;
-  if (!same_shape(q, k) || !same_shape(q, v) || !codes || !scales) return LX_ERR_INVALID;
+  if (!same_shape(q, k) || !same_shape(q, v) || !payload) return LX_ERR_INVALID;
   if (N < 1 || q->L % N != 0) return LX_ERR_INVALID;
-  if (!al16(codes) || !al16(scales)) return LX_ERR_ALIGN;
+  if (!al16(payload)) return LX_ERR_ALIGN;
   lx::UlyssesArgs a{};
   a.x[0] = rw(q);
   a.x[1] = rw(k);
   a.x[2] = rw(v);
-  a.codes = const_cast<uint8_t*>(codes);
-  a.scales = const_cast<float*>(scales);
+  a.payload = const_cast<uint8_t*>(payload);
+  long long rows_r;
+  ulysses_segment(q->B, q->H, q->L / N, q->D, 3, &rows_r, &a.sc_off, &a.seg);
   a.N = (int)N;
   a.B = (int)q->B;
   a.Hr = (int)q->H;
   a.Hc = (int)q->H;
   a.Lr = (int)(q->L / N);
-  a.rows = (long long)N * q->B * q->H * (q->L / N) * 3;
+  a.rows = (long long)N * rows_r;
   return launch_ulysses<lx::kUnpackQKV>(a, q->D, stream);
 }
 
-lx_status lx_ulysses_pack_o(const lx_bhld* o, int64_t N, uint8_t* codes, float* scales, cudaStream_t stream) {
+lx_status lx_ulysses_pack_o(const lx_bhld* o, int64_t N, uint8_t* payload, cudaStream_t stream) {
   lx_status st;
   if ((st = check_bhld(o)) != LX_OK) return st;
-  if (!codes || !scales || N < 1 || o->L % N != 0) return LX_ERR_INVALID;
-  if (!al16(codes) || !al16(scales)) return LX_ERR_ALIGN;
+  if (!payload || N < 1 || o->L % N != 0) return LX_ERR_INVALID;
+  if (!al16(payload)) return LX_ERR_ALIGN;
   lx::UlyssesArgs a{};
   a.x[0] = rw(o);
-  a.codes = codes;
-  a.scales = scales;
+  a.payload = payload;
+  long long rows_r;
+  ulysses_segment(o->B, o->H, o->L / N, o->D, 1, &rows_r, &a.sc_off, &a.seg);
   a.N = (int)N;
   a.B = (int)o->B;
   a.Hr = (int)o->H;
   a.Hc = (int)o->H;
   a.Lr = (int)(o->L / N);
-  a.rows = (long long)N * o->B * o->H * (o->L / N);
+  a.rows = (long long)N * rows_r;
   return launch_ulysses<lx::kPackO>(a, o->D, stream);
 }
 
-lx_status lx_ulysses_unpack_o(const uint8_t* codes, const float* scales, int64_t N, int64_t h0, int64_t hc,
-                              const lx_bhld* out, cudaStream_t stream) {
+lx_status lx_ulysses_unpack_o(const uint8_t* payload, int64_t N, int64_t h0, int64_t hc, const lx_bhld* out,
+                              cudaStream_t stream) {
   lx_status st;
   if ((st = check_bhld(out)) != LX_OK) return st;
-  if (!codes || !scales || N < 1 || out->H % N != 0 || h0 < 0 || hc < 1 || h0 + hc > out->H / N)
-    return LX_ERR_INVALID;
-  if (!al16(codes) || !al16(scales)) return LX_ERR_ALIGN;
+  if (!payload || N < 1 || out->H % N != 0 || h0 < 0 || hc < 1 || h0 + hc > out->H / N) return LX_ERR_INVALID;
+  if (!al16(payload)) return LX_ERR_ALIGN;
   lx::UlyssesArgs a{};
   a.x[0] = rw(out);
-  a.codes = const_cast<uint8_t*>(codes);
-  a.scales = const_cast<float*>(scales);
+  a.payload = const_cast<uint8_t*>(payload);
+  long long rows_r;
+  ulysses_segment(out->B, hc, out->L, out->D, 1, &rows_r, &a.sc_off, &a.seg);
   a.N = (int)N;
   a.B = (int)out->B;
   a.Hr = (int)(out->H / N);
   a.Hc = (int)hc;
   a.h0 = (int)h0;
   a.Lr = (int)out->L;
-  a.rows = (long long)N * out->B * hc * out->L;
+  a.rows = (long long)N * rows_r;
   return launch_ulysses<lx::kUnpackO>(a, out->D, stream);
 }
 

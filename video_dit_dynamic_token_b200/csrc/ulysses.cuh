@@ -10,11 +10,14 @@
 // values, s = absmax/448 (1 for an all-zero row), code = E4M3_rn_satfinite(
 // fl32(x * fl32(448/absmax))); the receiver takes bf16(fl32(decode * s)).
 //
-// Buffers (dense, row-major):
-//   Q/K/V payload to rank n: codes [N][B][Hc][Lr][3][D], scales [N][B][Hc][Lr][3]
-//   output payload to rank n: codes [N][B][Hc][Lr][D],   scales [N][B][Hc][Lr]
+// One payload buffer per exchange, one segment of `seg` bytes per destination
+// rank n (so that a single all-to-all with equal splits moves it):
+//   Q/K/V segment: codes [B][Hc][Lr][3][D] uint8, then at byte offset sc_off
+//                  scales [B][Hc][Lr][3] fp32
+//   output segment: codes [B][Hc][Lr][D], then scales [B][Hc][Lr]
 // where Hc is the number of heads of one exchange (a chunk of the Hr heads of
-// each destination, starting at head h0 of its range).
+// each destination, starting at head h0 of its range); sc_off and seg are the
+// code and scale byte counts rounded up to 16.
 #pragma once
 #include <cuda_bf16.h>
 #include <cstdint>
@@ -32,10 +35,11 @@ enum UlyssesMode : int { kPackQKV = 0, kPackO = 1, kUnpackQKV = 2, kUnpackO = 3 
 struct UlyssesArgs {
   BhldRW x[3];      // pack QKV: q, k, v shards [B, H, Lr, D]; unpack QKV: q, k, v chunks [B, Hc, L, D];
                     // pack O: o chunk [B, Hc, L, D]; unpack O: out shard [B, H, Lr, D]
-  uint8_t* codes;
-  float* scales;
+  uint8_t* payload;
+  long long seg;     // bytes per destination segment
+  long long sc_off;  // byte offset of the scales within a segment
   int N, B, Hr, Hc, h0, Lr;
-  long long rows;   // rows of the payload
+  long long rows;    // rows of the payload (all segments)
 };
 
 // Four consecutive E4M3 codes (lowest byte first) to floats.
@@ -70,7 +74,10 @@ __global__ void __launch_bounds__(256) ulysses_rows_kernel(UlyssesArgs a) {
   const int b = (ny / a.Hc) % a.B;
   const int n = ny / (a.Hc * a.B);
   const int slice_rows = a.Lr * X;
-  const long long slice0 = (long long)ny * slice_rows;  // payload row of the slice's first row
+  // the slice's first row within destination n's segment
+  const long long slice0 = (long long)(ny - n * a.B * a.Hc) * slice_rows;
+  uint8_t* codes = a.payload + (long long)n * a.seg;
+  float* scales = reinterpret_cast<float*>(codes + a.sc_off);
   const int base = blockIdx.x * G * kUlyPasses;
   __nv_bfloat16* xr[kUlyPasses];
   long long pr[kUlyPasses];
@@ -117,8 +124,8 @@ __global__ void __launch_bounds__(256) ulysses_rows_kernel(UlyssesArgs a) {
       const uint32_t c0 = e4m3x4(y[0], y[1], y[2], y[3]);
       const uint32_t c1 = e4m3x4(y[4], y[5], y[6], y[7]);
       if (live[i]) {
-        *reinterpret_cast<uint2*>(a.codes + pr[i] * D + c * 8) = make_uint2(c0, c1);
-        if (c == 0) a.scales[pr[i]] = m > 0.f ? __fdiv_rn(m, 448.0f) : 1.0f;
+        *reinterpret_cast<uint2*>(codes + pr[i] * D + c * 8) = make_uint2(c0, c1);
+        if (c == 0) scales[pr[i]] = m > 0.f ? __fdiv_rn(m, 448.0f) : 1.0f;
       }
     }
   } else {
@@ -126,8 +133,8 @@ __global__ void __launch_bounds__(256) ulysses_rows_kernel(UlyssesArgs a) {
     float s[kUlyPasses];
 #pragma unroll
     for (int i = 0; i < kUlyPasses; ++i) {
-      cw[i] = live[i] ? *reinterpret_cast<const uint2*>(a.codes + pr[i] * D + c * 8) : make_uint2(0, 0);
-      s[i] = live[i] ? a.scales[pr[i]] : 0.f;
+      cw[i] = live[i] ? *reinterpret_cast<const uint2*>(codes + pr[i] * D + c * 8) : make_uint2(0, 0);
+      s[i] = live[i] ? scales[pr[i]] : 0.f;
     }
 #pragma unroll
     for (int i = 0; i < kUlyPasses; ++i) {

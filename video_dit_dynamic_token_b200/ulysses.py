@@ -5,9 +5,10 @@ contiguous part of the token sequence; an all-to-all moves Q, K and V (one FP8
 payload) to head-sharded form, each GPU runs the attention of its heads, and a
 second all-to-all (FP8 again) brings the output back to sequence-sharded form;
 the exchange runs per head chunk, the next chunk in flight while the current
-one computes.  The payload layouts and the FP8 rule are those of the
-lx_ulysses_* calls (include/lx_sparse_attn.h); the collectives are
-torch.distributed all-to-alls with equal splits (NCCL on the GPU).
+one computes.  Each exchange is one all-to-all with equal splits (NCCL on the
+GPU) over one byte payload of N segments, each segment holding a
+destination's FP8 codes and then their fp32 scales; the layout and the FP8
+rule are those of the lx_ulysses_* calls (include/lx_sparse_attn.h).
 
 The per-step operations are passed in as `UlyssesOps`; the default runs the
 CUDA kernels and lx_sparse_attn.  Nothing here computes on the host.
@@ -24,34 +25,61 @@ import torch.distributed as dist
 from . import _abi, _check, _ptr, _stream, bhld, lx_sparse_attn
 
 
+# ---------------------------------------------------------------- payload layout
+def segment_layout(B, hc, Lr, D, X):
+    """(rows, byte offset of the scales, bytes) of one destination's segment:
+    codes uint8 [B, hc, Lr, X, D], then from the 16-byte rounded code size the
+    scales fp32 [B, hc, Lr, X], the segment rounded up to 16 bytes
+    (lx_ulysses_segment_bytes gives the same size)."""
+    rows = B * hc * Lr * X
+    sc_off = (rows * D + 15) // 16 * 16
+    return rows, sc_off, sc_off + (rows * 4 + 15) // 16 * 16
+
+
+def new_payload(N, B, hc, Lr, D, X, device):
+    return torch.empty((N, segment_layout(B, hc, Lr, D, X)[2]), dtype=torch.uint8, device=device)
+
+
+def payload_views(payload, B, hc, Lr, D, X):
+    """The codes [N, B, hc, Lr, (X,) D] and scales [N, B, hc, Lr, (X)] inside a
+    payload [N, seg] (views, no copy; the X axis is dropped for X = 1)."""
+    N = payload.shape[0]
+    rows, sc_off, _ = segment_layout(B, hc, Lr, D, X)
+    shape = (N, B, hc, Lr, X) if X > 1 else (N, B, hc, Lr)
+    codes = payload[:, :rows * D].view(*shape, D)
+    scales = payload[:, sc_off:sc_off + rows * 4].view(torch.float32).view(*shape)
+    return codes, scales
+
+
 # ---------------------------------------------------------------- CUDA operations
-def pack_qkv(qv, kv, vv, N, h0, hc, codes, scales, stream=None):
-    """qv, kv, vv: [B, H, Lr, D] views of this rank's shard -> payload buffers."""
+def pack_qkv(qv, kv, vv, N, h0, hc, payload, stream=None):
+    """qv, kv, vv: [B, H, Lr, D] views of this rank's shard -> payload [N, seg]."""
     lib = _abi.load()
     q, k, v = bhld(qv), bhld(kv), bhld(vv)
-    _check(lib.lx_ulysses_pack_qkv(ctypes.byref(q), ctypes.byref(k), ctypes.byref(v), N, h0, hc, _ptr(codes),
-                                   _ptr(scales), _stream(stream)), "lx_ulysses_pack_qkv")
+    _check(lib.lx_ulysses_pack_qkv(ctypes.byref(q), ctypes.byref(k), ctypes.byref(v), N, h0, hc, _ptr(payload),
+                                   _stream(stream)), "lx_ulysses_pack_qkv")
 
 
-def unpack_qkv(codes, scales, N, qh, kh, vh, stream=None):
-    """Received payload -> q, k, v [B, hc, L, D]."""
+def unpack_qkv(payload, N, qh, kh, vh, stream=None):
+    """Received payload [N, seg] -> q, k, v [B, hc, L, D]."""
     lib = _abi.load()
     q, k, v = bhld(qh), bhld(kh), bhld(vh)
-    _check(lib.lx_ulysses_unpack_qkv(_ptr(codes), _ptr(scales), N, ctypes.byref(q), ctypes.byref(k), ctypes.byref(v),
+    _check(lib.lx_ulysses_unpack_qkv(_ptr(payload), N, ctypes.byref(q), ctypes.byref(k), ctypes.byref(v),
                                      _stream(stream)), "lx_ulysses_unpack_qkv")
 
 
-def pack_o(oh, N, codes, scales, stream=None):
+def pack_o(oh, N, payload, stream=None):
+    """Attention output [B, hc, L, D] -> payload [N, seg] (segment n: rank n's tokens)."""
     lib = _abi.load()
     o = bhld(oh)
-    _check(lib.lx_ulysses_pack_o(ctypes.byref(o), N, _ptr(codes), _ptr(scales), _stream(stream)), "lx_ulysses_pack_o")
+    _check(lib.lx_ulysses_pack_o(ctypes.byref(o), N, _ptr(payload), _stream(stream)), "lx_ulysses_pack_o")
 
 
-def unpack_o(codes, scales, N, h0, hc, outv, stream=None):
+def unpack_o(payload, N, h0, hc, outv, stream=None):
     """Received output payload -> heads of this rank's shard view outv [B, H, Lr, D]."""
     lib = _abi.load()
     o = bhld(outv)
-    _check(lib.lx_ulysses_unpack_o(_ptr(codes), _ptr(scales), N, h0, hc, ctypes.byref(o), _stream(stream)),
+    _check(lib.lx_ulysses_unpack_o(_ptr(payload), N, h0, hc, ctypes.byref(o), _stream(stream)),
            "lx_ulysses_unpack_o")
 
 
@@ -100,32 +128,28 @@ def ulysses_sparse_attn(q, k, v, keep, mode="int8fp8", group=None, n_chunks=2, o
     chunks = head_chunks(Hr, n_chunks)
 
     def start_qkv(h0, hc):
-        sc = torch.empty((N, B, hc, Lr, 3, D), dtype=torch.uint8, device=dev)
-        ss = torch.empty((N, B, hc, Lr, 3), dtype=torch.float32, device=dev)
-        ops.pack_qkv(qv, kv, vv, N, h0, hc, sc, ss)
-        rc, rs = torch.empty_like(sc), torch.empty_like(ss)
-        return rc, rs, [_exchange(rc, sc, group), _exchange(rs, ss, group)], (sc, ss)
+        send = new_payload(N, B, hc, Lr, D, 3, dev)
+        ops.pack_qkv(qv, kv, vv, N, h0, hc, send)
+        recv = torch.empty_like(send)
+        return recv, _exchange(recv, send, group), send
 
     pending_out = []
     nxt = start_qkv(*chunks[0])
     for i, (h0, hc) in enumerate(chunks):
-        rc, rs, works, _keep_alive = nxt
+        recv, work, _keep_alive = nxt
         if i + 1 < len(chunks):       # the next chunk's payload travels while this one computes
             nxt = start_qkv(*chunks[i + 1])
-        for w in works:
-            if w is not None:
-                w.wait()
+        if work is not None:
+            work.wait()
         qh, kh, vh = (torch.empty((B, hc, L, D), dtype=torch.bfloat16, device=dev) for _ in range(3))
-        ops.unpack_qkv(rc, rs, N, qh, kh, vh)
+        ops.unpack_qkv(recv, N, qh, kh, vh)
         oh = attention(qh, kh, vh)
-        oc = torch.empty((N, B, hc, Lr, D), dtype=torch.uint8, device=dev)
-        os_ = torch.empty((N, B, hc, Lr), dtype=torch.float32, device=dev)
-        ops.pack_o(oh, N, oc, os_)
-        roc, ros = torch.empty_like(oc), torch.empty_like(os_)
-        pending_out.append((h0, hc, roc, ros, [_exchange(roc, oc, group), _exchange(ros, os_, group)], (oc, os_)))
-    for h0, hc, roc, ros, works, _keep_alive in pending_out:
-        for w in works:
-            if w is not None:
-                w.wait()
-        ops.unpack_o(roc, ros, N, h0, hc, outv)
+        send_o = new_payload(N, B, hc, Lr, D, 1, dev)
+        ops.pack_o(oh, N, send_o)
+        recv_o = torch.empty_like(send_o)
+        pending_out.append((h0, hc, recv_o, _exchange(recv_o, send_o, group), send_o))
+    for h0, hc, recv_o, work, _keep_alive in pending_out:
+        if work is not None:
+            work.wait()
+        ops.unpack_o(recv_o, N, h0, hc, outv)
     return out
