@@ -44,6 +44,14 @@ ATTN_KERNEL = {"int8fp8": ("sparse_attn_paired_kernel", ("attn.cuh", "attn_paire
 # capture, keyed by the SHA-256 of the kernel sources it was taken on: when
 # they change the key no longer matches and the line reports null.
 ATTN_DRAM_BYTES = {   # {sha256 of the mode's sources: (bytes per full 720p launch, how it was taken)}
+    "5e535f16af26913e923f8e56615036cb11ac3999d4bf110eca695ccf31af8166":
+        (5 * (236.936960e6 + 126.448640e6),
+         "ncu dram__bytes_read.sum + dram__bytes_write.sum of the 8-head 720p launch x 5 (traffic grows with the "
+         "heads)"),
+    "247dd9af093a5ac2507a8ddc7203d69c4d870f132de6b26845a01fc7a98d16dc":
+        (5 * (471.053312e6 + 141.109760e6),
+         "ncu dram__bytes_read.sum + dram__bytes_write.sum of the 8-head 720p BF16 launch x 5 (traffic grows with "
+         "the heads)"),
 }
 
 # Dense MACs per clock per SM of one tcgen05 kind::i8 / kind::f8f6f4 M=128 MMA
