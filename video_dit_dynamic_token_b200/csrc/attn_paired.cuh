@@ -22,8 +22,10 @@
 // before it writes P(c).
 //
 // Roles (6 warps): warp 0 = TMA producer (Q once; K blocks of both streams, a
-// pair of steps at a time, into one stage; V blocks into a 2-stage ring);
-// warp 1 = TMEM allocator + MMA issuer; warps 2..5 = softmax / correction /
+// pair of steps at a time, into one stage, reused once that pair's S is
+// complete; V blocks into a 2-stage ring), one thread; warp 1 = TMEM allocator
+// + MMA issuer, a warp-wide loop whose waits are voted and whose MMAs one
+// elected lane issues; warps 2..5 = softmax / correction /
 // epilogue, one thread per (stream, row): thread t of warp w reads TMEM lane
 // 32*(w%4) + t, i.e. row 16*(w%4) + t%16 of stream t/16.
 //
@@ -71,7 +73,7 @@ __global__ void __launch_bounds__(192, I8 ? 2 : 1)
   using C = AttnPairCfg<D, I8>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  __shared__ uint64_t bar_q, bar_kfull, bar_kempty, bar_vfull[C::VSTAGE],
+  __shared__ uint64_t bar_q, bar_kfull, bar_vfull[C::VSTAGE],
       bar_vempty[C::VSTAGE], bar_sfull, bar_sfree, bar_pfull, bar_odone, bar_drain;
   __shared__ uint32_t tmem_slot;
   __shared__ volatile int abort_flag;
@@ -92,7 +94,6 @@ __global__ void __launch_bounds__(192, I8 ? 2 : 1)
   if (threadIdx.x == 0) {
     mbar_init(&bar_q, 1);
     mbar_init(&bar_kfull, 1);
-    mbar_init(&bar_kempty, 1);
     for (int s = 0; s < C::VSTAGE; ++s) {
       mbar_init(&bar_vfull[s], 1);
       mbar_init(&bar_vempty[s], 1);
@@ -148,7 +149,7 @@ __global__ void __launch_bounds__(192, I8 ? 2 : 1)
           // K blocks of steps c and c+1 (both streams) into the pair stage,
           // once S of the previous pair has read it
           const int p = c >> 1;
-          ok = p == 0 || mbar_wait(&bar_kempty, (p - 1) & 1, &abort_flag, prm.limit_ns);
+          ok = p == 0 || mbar_wait(&bar_sfull, (p - 1) & 1, &abort_flag, prm.limit_ns);
           if (!ok) break;
           const int nb = (c + 1 < n) ? 2 : 1;
           mbar_arrive_expect_tx(&bar_kfull, (uint32_t)nb * kv_tx);
@@ -186,8 +187,9 @@ __global__ void __launch_bounds__(192, I8 ? 2 : 1)
         mbar_wait(&bar_vfull[cc % C::VSTAGE], (cc / C::VSTAGE) & 1, &never_abort, prm.limit_ns);
     }
   } else if (warp == 1) {
-    // ================= MMA issuer =================
-    if (lane == 0) {
+    // ================= MMA issuer (warp-wide loop, one elected lane issues) =================
+    const bool leader = elect_one();
+    {
       // Descriptors of stage 0 / stream A; a shared-memory descriptor's start
       // address sits in its low 14 bits (address >> 4, below 256 KB), so other
       // stages, streams and K steps are plain additions of (offset >> 4).
@@ -195,7 +197,7 @@ __global__ void __launch_bounds__(192, I8 ? 2 : 1)
       const uint64_t dK = smem_desc(smem_u32(sm + C::OFF_K), 16, 8 * C::ATOM, C::SW_QKV);
       const uint64_t dP = smem_desc(smem_u32(sm + C::OFF_P), 16, 8 * C::P_ROWB, C::SW_P);
       const uint64_t dV = smem_desc(smem_u32(sm + C::OFF_V), 64 * C::ATOM, 8 * C::ATOM, C::SW_QKV);
-      bool ok = mbar_wait(&bar_q, 0, &abort_flag, prm.limit_ns);
+      bool ok = warp_wait(&bar_q, 0, &abort_flag, prm.limit_ns);
       tc_fence_after();
       // Iteration c issues S of pair p+1 (when c = 2p+1; pair 0 goes first)
       // and then P(c).V.  S of pair p+1 needs the softmax to have read both
@@ -203,10 +205,11 @@ __global__ void __launch_bounds__(192, I8 ? 2 : 1)
       for (int c = -1; ok && c < n; ++c) {
         const int p = (c + 1) >> 1;  // the pair whose S is issued in this iteration
         if ((c & 1) != 0 && p < npairs) {  // c = -1, 1, 3, ...
-          ok = mbar_wait(&bar_kfull, p & 1, &abort_flag, prm.limit_ns) &&
-               mbar_wait(&bar_sfree, p & 1, &abort_flag, prm.limit_ns);
+          ok = warp_wait(&bar_kfull, p & 1, &abort_flag, prm.limit_ns) &&
+               warp_wait(&bar_sfree, p & 1, &abort_flag, prm.limit_ns);
           if (!ok) break;
           tc_fence_after();
+          if (leader) {
 #pragma unroll
           for (int s = 0; s < 2; ++s) {
             if (s == 1 && !has1) break;
@@ -220,15 +223,17 @@ __global__ void __launch_bounds__(192, I8 ? 2 : 1)
                                               (I8 || kk > 0) ? 1u : 0u);
             }
           }
-          mma_commit(&bar_sfull);
-          mma_commit(&bar_kempty);
+          mma_commit(&bar_sfull);   // S complete: also frees the K pair stage
+          }
+          __syncwarp();
         }
         if (c >= 0) {
           const int vs = c % C::VSTAGE;
-          ok = mbar_wait(&bar_vfull[vs], (c / C::VSTAGE) & 1, &abort_flag, prm.limit_ns) &&
-               mbar_wait(&bar_pfull, c & 1, &abort_flag, prm.limit_ns);
+          ok = warp_wait(&bar_vfull[vs], (c / C::VSTAGE) & 1, &abort_flag, prm.limit_ns) &&
+               warp_wait(&bar_pfull, c & 1, &abort_flag, prm.limit_ns);
           if (!ok) break;
           tc_fence_after();
+          if (leader) {
           const uint64_t dVs = dV + (uint64_t)((vs * 2 * C::KV_BYTES) >> 4);
 #pragma unroll
           for (int s = 0; s < 2; ++s) {
@@ -243,15 +248,20 @@ __global__ void __launch_bounds__(192, I8 ? 2 : 1)
           }
           mma_commit(&bar_odone);
           mma_commit(&bar_vempty[vs]);
+          }
+          __syncwarp();
         }
       }
-      if (!ok) {
+      if (!ok && leader) {
         abort_flag = 1;
         report_error(-6);
       }
       // drain: all issued MMAs complete before TMEM is released
-      mma_commit(&bar_drain);
-      mbar_wait(&bar_drain, 0, &never_abort, prm.limit_ns);
+      if (leader) {
+        mma_commit(&bar_drain);
+        mbar_wait(&bar_drain, 0, &never_abort, prm.limit_ns);
+      }
+      __syncwarp();
     }
   } else {
     // ================= softmax / correction / epilogue =================
