@@ -414,18 +414,24 @@ __global__ void __launch_bounds__(192, I8 ? 2 : 1)
           const float f = need_rescale ? alpha : 1.f;
           const uint64_t f2 = f2pack(f, f);
 #pragma unroll
-          for (int cc = 0; cc < D; cc += 32) {
-            uint32_t o[32];
-            tmem_ld32(lane_addr + C::O_COL + cc, o);
+          for (int cc = 0; cc < D; cc += 64) {   // two 32-column loads in flight per round trip
+            uint32_t o[2][32];
+            tmem_ld32(lane_addr + C::O_COL + cc, o[0]);
+            if (cc + 32 < D) tmem_ld32(lane_addr + C::O_COL + cc + 32, o[1]);
             tmem_wait_ld();
 #pragma unroll
-            for (int i = 0; i < 32; i += 2) {
-              float a, b;
-              f2unpack(mul2(f2pack(__uint_as_float(o[i]), __uint_as_float(o[i + 1])), f2), a, b);
-              o[i] = __float_as_uint(a);
-              o[i + 1] = __float_as_uint(b);
+            for (int hh = 0; hh < 2; ++hh) {
+              if (cc + 32 * hh < D) {
+#pragma unroll
+                for (int i = 0; i < 32; i += 2) {
+                  float a, b;
+                  f2unpack(mul2(f2pack(__uint_as_float(o[hh][i]), __uint_as_float(o[hh][i + 1])), f2), a, b);
+                  o[hh][i] = __float_as_uint(a);
+                  o[hh][i + 1] = __float_as_uint(b);
+                }
+                tmem_st32(lane_addr + C::O_COL + cc + 32 * hh, o[hh]);
+              }
             }
-            tmem_st32(lane_addr + C::O_COL + cc, o);
           }
           tmem_wait_st();
         }
