@@ -44,8 +44,8 @@ ATTN_KERNEL = {"int8fp8": ("sparse_attn_paired_kernel", ("attn.cuh", "attn_paire
 # capture, keyed by the SHA-256 of the kernel sources it was taken on: when
 # they change the key no longer matches and the line reports null.
 ATTN_DRAM_BYTES = {   # {sha256 of the mode's sources: (bytes per full 720p launch, how it was taken)}
-    "522677a7f042f41b51aa9fe06306ae166aaad346df2a194189a699c4d92b7f6f":
-        (5 * (237.637632e6 + 126.666752e6),
+    "879e6bb5ea0b0ae55928d3858cae030564a0462f2718dfe262a4a06f3fecd646":
+        (5 * (236.927744e6 + 126.024448e6),
          "ncu dram__bytes_read.sum + dram__bytes_write.sum of the 8-head 720p launch x 5 (traffic grows with the "
          "heads)"),
     "247dd9af093a5ac2507a8ddc7203d69c4d870f132de6b26845a01fc7a98d16dc":
