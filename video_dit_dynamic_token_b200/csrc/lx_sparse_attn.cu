@@ -204,22 +204,13 @@ lx_status launch_quant_v(const lx_bhld* V, uint8_t* vc, float* vs, uint32_t* ama
   return launch_status();
 }
 
-// INT8/FP8 attention: the paired-S kernel (attn_paired.cuh)
+// Kernel arguments shared by both attention kernels.
 template <int D>
-lx_status launch_attn_paired(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const lx_plan* plan,
-                             const lx_bhld* O, const float* qs, const float* ks, const float* vs, cudaStream_t s) {
-  using C = lx::AttnPairCfg<D, true>;
-  const int64_t nB = plan->nB;
-  // the two kept lists follow the tiles
-  const size_t smem = 1024 + C::OFF_IDX + 2 * sizeof(int32_t) * (size_t)plan->k;
-  if (smem > 227 * 1024) return LX_ERR_UNSUPPORTED;
-  if (cudaFuncSetAttribute(lx::sparse_attn_paired_kernel<D, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           (int)smem) != cudaSuccess)
-    return LX_ERR_CUDA;
+lx::AttnParams attn_params(const lx_plan* plan, const lx_bhld* O, const float* qs, const float* ks, const float* vs) {
   lx::AttnParams p;
   p.idx = plan->idx;
   p.k = (int)plan->k;
-  p.nB = (int)nB;
+  p.nB = (int)plan->nB;
   p.L = (int)plan->L;
   p.H = (int)plan->H;
   p.o = reinterpret_cast<__nv_bfloat16*>(O->data);
@@ -231,9 +222,27 @@ lx_status launch_attn_paired(const CUtensorMap& mq, const CUtensorMap& mk, const
   p.sv = vs;
   p.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)D));
   p.limit_ns = kWaitLimitNs;
-  // one CTA per (pair of query blocks, b*h), head-major so that a head's K/V stays in L2
-  dim3 grid((unsigned)((nB + 1) / 2), (unsigned)(plan->B * plan->H));
-  lx::sparse_attn_paired_kernel<D, true><<<grid, 192, smem, s>>>(mq, mk, mv, p);
+  return p;
+}
+
+// one CTA per (pair of query blocks, b*h), head-major so that a head's K/V stays in L2
+inline dim3 attn_grid(const lx_plan* plan) {
+  return dim3((unsigned)((plan->nB + 1) / 2), (unsigned)(plan->B * plan->H));
+}
+
+// INT8/FP8 attention: the paired-S kernel (attn_paired.cuh)
+template <int D>
+lx_status launch_attn_paired(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const lx_plan* plan,
+                             const lx_bhld* O, const float* qs, const float* ks, const float* vs, cudaStream_t s) {
+  using C = lx::AttnPairCfg<D, true>;
+  // the two kept lists follow the tiles
+  const size_t smem = 1024 + C::OFF_IDX + 2 * sizeof(int32_t) * (size_t)plan->k;
+  if (smem > 227 * 1024) return LX_ERR_UNSUPPORTED;
+  if (cudaFuncSetAttribute(lx::sparse_attn_paired_kernel<D, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)smem) != cudaSuccess)
+    return LX_ERR_CUDA;
+  lx::sparse_attn_paired_kernel<D, true><<<attn_grid(plan), 192, smem, s>>>(mq, mk, mv,
+                                                                           attn_params<D>(plan, O, qs, ks, vs));
   return launch_status();
 }
 
@@ -242,31 +251,14 @@ template <int D, bool I8>
 lx_status launch_attn(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const lx_plan* plan,
                       const lx_bhld* O, const float* qs, const float* ks, const float* vs, cudaStream_t s) {
   using C = lx::AttnCfg<D, I8>;
-  const int64_t nB = plan->nB;
   // the two kept lists and their K scales follow the tiles
   const size_t smem = 1024 + C::OFF_IDX + 16 * (size_t)plan->k;
   if (smem > 227 * 1024) return LX_ERR_UNSUPPORTED;
   if (cudaFuncSetAttribute(lx::sparse_attn_kernel<D, I8>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
       cudaSuccess)
     return LX_ERR_CUDA;
-  lx::AttnParams p;
-  p.idx = plan->idx;
-  p.k = (int)plan->k;
-  p.nB = (int)nB;
-  p.L = (int)plan->L;
-  p.H = (int)plan->H;
-  p.o = reinterpret_cast<__nv_bfloat16*>(O->data);
-  p.osB = O->sB;
-  p.osH = O->sH;
-  p.osL = O->sL;
-  p.sq = qs;
-  p.sk = ks;
-  p.sv = vs;
-  p.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)D));
-  p.limit_ns = kWaitLimitNs;
-  // one CTA per (pair of query blocks, b*h), head-major so that a head's K/V stays in L2
-  dim3 grid((unsigned)((nB + 1) / 2), (unsigned)(plan->B * plan->H));
-  lx::sparse_attn_kernel<D, I8><<<grid, C::THREADS, smem, s>>>(mq, mk, mv, p);
+  lx::sparse_attn_kernel<D, I8><<<attn_grid(plan), C::THREADS, smem, s>>>(mq, mk, mv,
+                                                                          attn_params<D>(plan, O, qs, ks, vs));
   return launch_status();
 }
 
