@@ -201,12 +201,6 @@ constexpr int kScoreWarps = 8;
 constexpr int kBuckets = 128;
 constexpr int kMaxChunks = 17;  // 128-score chunks of the longest row (nB <= 2176)
 
-__device__ __forceinline__ uint32_t lanemask_lt() {
-  uint32_t m;
-  asm("mov.u32 %0, %%lanemask_lt;" : "=r"(m));
-  return m;
-}
-
 // Bucket of a score: (s - mn) * scale clamped to [0, 127] and rounded to the
 // nearest integer by adding 1.5 * 2^23 (whose float spacing is 1), then read
 // from the bits.  Non-decreasing in s.  For a finite row s - mn >= 0; a NaN
@@ -327,8 +321,9 @@ __device__ int select_row(float* s, int nB, int k, int* hist, float* cand_s, int
     // members of bucket bt, ranked by (score desc, index asc)
     const int c = hist[bt];
     if (c <= kCandCap) {
-      const uint32_t lt = lanemask_lt();
-      int base = 0;
+      // membership words: word 4c + e is the ballot of score e of chunk c
+      // (ids 32 (4c + e) + lane); lane l keeps words l, l + 32 and l + 64
+      uint32_t wk[3] = {0u, 0u, 0u};
 #pragma unroll
       for (int ch = 0; ch < kMaxChunks; ++ch) {
         if (ch >= nC) break;
@@ -338,14 +333,32 @@ __device__ int select_row(float* s, int nB, int k, int* hist, float* cand_s, int
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
           const uint32_t b = __ballot_sync(0xffffffffu, (m >> e) & 1u);
-          if ((m >> e) & 1u) {
-            const int pos = base + __popc(b & lt);
-            const int j = 128 * ch + 32 * e + lane;
-            cand_s[pos] = s[j];
-            cand_j[pos] = j;
-          }
-          base += __popc(b);
+          if (lane == ((4 * ch + e) & 31)) wk[(4 * ch + e) >> 5] = b;
         }
+      }
+      // each lane expands its words, ascending, at the offset given by the
+      // popcounts of the words before it
+      int base = 0;
+#pragma unroll
+      for (int g = 0; g < 3; ++g) {
+        if (32 * g >= nW) break;
+        uint32_t mm = wk[g];
+        const int cnt = __popc(mm);
+        int incl = cnt;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+          const int v = __shfl_up_sync(0xffffffffu, incl, off);
+          if (lane >= off) incl += v;
+        }
+        int pos = base + incl - cnt;
+        while (mm) {
+          const int j = 32 * (32 * g + lane) + __ffs(mm) - 1;
+          mm &= mm - 1;
+          cand_s[pos] = s[j];
+          cand_j[pos] = j;
+          ++pos;
+        }
+        base += __shfl_sync(0xffffffffu, incl, 31);
       }
       __syncwarp();
       for (int i = lane; i < c; i += 32) {
@@ -381,11 +394,8 @@ __device__ int select_row(float* s, int nB, int k, int* hist, float* cand_s, int
     }
     __syncwarp();
   }
-  // emit ascending ids into the row buffer; mask word 4c + e is the ballot of
-  // score e of the lanes and replaces selbits word 4c + e once it has been read
-  int* ids = reinterpret_cast<int*>(s);
-  const uint32_t lt = lanemask_lt();
-  int written = 0;
+  // the mask words first: word 4c + e is the ballot of score e of the lanes in
+  // chunk c, and replaces selbits word 4c + e once every lane has read it
 #pragma unroll
   for (int ch = 0; ch < kMaxChunks; ++ch) {
     if (ch >= nC) break;
@@ -408,18 +418,31 @@ __device__ int select_row(float* s, int nB, int k, int* hist, float* cand_s, int
     }
     const uint32_t b0 = __ballot_sync(0xffffffffu, sel & 1u), b1 = __ballot_sync(0xffffffffu, sel & 2u);
     const uint32_t b2 = __ballot_sync(0xffffffffu, sel & 4u), b3 = __ballot_sync(0xffffffffu, sel & 8u);
-    const int p0 = __popc(b0), p1 = __popc(b1), p2 = __popc(b2);
-    const int j = 128 * ch + lane;
-    if (sel) {
-      int pos;
-      if ((sel & 1u) && (pos = written + __popc(b0 & lt)) < k) ids[pos] = j;
-      if ((sel & 2u) && (pos = written + p0 + __popc(b1 & lt)) < k) ids[pos] = j + 32;
-      if ((sel & 4u) && (pos = written + p0 + p1 + __popc(b2 & lt)) < k) ids[pos] = j + 64;
-      if ((sel & 8u) && (pos = written + p0 + p1 + p2 + __popc(b3 & lt)) < k) ids[pos] = j + 96;
-    }
-    // every lane's selbits reads for this chunk fed the ballots above
     if (lane < 4 && 4 * ch + lane < nW) selbits[4 * ch + lane] = lane == 0 ? b0 : (lane == 1 ? b1 : (lane == 2 ? b2 : b3));
-    written += p0 + p1 + p2 + __popc(b3);
+  }
+  __syncwarp();
+  // then the ids, ascending, into the row buffer (no longer read): lane l
+  // expands word w0 + l at the offset given by the popcounts of the words before it
+  int* ids = reinterpret_cast<int*>(s);
+  int written = 0;
+  for (int w0 = 0; w0 < nW; w0 += 32) {
+    const int w = w0 + lane;
+    uint32_t m = w < nW ? selbits[w] : 0u;
+    const int cnt = __popc(m);
+    int incl = cnt;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int v = __shfl_up_sync(0xffffffffu, incl, off);
+      if (lane >= off) incl += v;
+    }
+    int pos = written + incl - cnt;
+    while (m) {
+      const int b = __ffs(m) - 1;
+      m &= m - 1;
+      if (pos < k) ids[pos] = 32 * w + b;
+      ++pos;
+    }
+    written += __shfl_sync(0xffffffffu, incl, 31);
   }
   __syncwarp();
   const int n_out = min(written, k);
